@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""CSA2 decode-step benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference] [--config C]
+
+One step = the whole decode hot path over one batch: (append,) index and the
+attends of every layer of the workload's schedule.  Default workload: the
+reuse group at 1M context (4 requests x 1,048,576 entries, Full + 3 Reuse +
+Reindex + 3 Reuse, 64 heads).  The step is captured once in a CUDA graph and
+replayed; each timed replay is bracketed by CUDA events, with a 256 MB write
+between replays to flush L2.  Under torchrun every rank runs its own replica
+(weak scaling) and the slowest rank's time counts.
+
+--impl reference times the CPU oracle (plain C, one thread) on the host,
+round-robin over the stages of one request's step, and reports the same
+metric; it runs on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "CSA2 decode queries/s at 1M ctx; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def algorithmic_bytes(w: synth.Workload) -> dict:
+    """Bytes the step must move, per the layout (per request, summed):
+    index  FULL: ceil(N/8)*128 [if > 2048 blocks] + min(N,16384)*128 + 16384*4
+           FLAT: N*128;  REINDEX: 16384*(128+4)
+    attend per layer: 512*288 + min(n_tok,128)*516 + 2*H*512*2 + 512*4
+    append: m*(641)*4 + 416 + 128 + 7*128 + m*516."""
+    tot = {"index": 0, "block_summaries": 0, "attend": 0, "append": 0}
+    for b in range(w.batch):
+        T = w.n_tok[b] + w.n_new[b]
+        N = T // w.m[b]
+        nb = -(-N // 8)
+        for mode in w.layers:
+            if mode == "full":
+                if w.index == "flat":
+                    tot["index"] += N * 128
+                else:
+                    summ = nb * 128 if nb > 2048 else 0
+                    tot["block_summaries"] += nb * 128
+                    tot["index"] += summ + min(N, 16384) * 128 + 16384 * 4
+            elif mode == "reindex":
+                tot["index"] += 16384 * (128 + 4)
+            tot["attend"] += 512 * 288 + min(T, 128) * 516 + 2 * w.heads * 512 * 2 + 512 * 4
+        if w.append:
+            m = w.m[b]
+            tot["append"] += m * 641 * 4 + 416 + 128 + 7 * 128 + m * 516
+    tot["step"] = tot["index"] + tot["attend"] + tot["append"]
+    return tot
+
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) side
+class OracleQuery:
+    """The oracle's decode step for one request of workload w, split into
+    stage units so it can be timed in bounded slices."""
+
+    CHUNK = 4096
+
+    def __init__(self, w: synth.Workload, b: int = 0):
+        import oracle
+        self.o = oracle
+        self.w, self.b = w, b
+        T = w.n_tok[b]
+        m = w.m[b]
+        chan = synth.channel_scale(w)
+        n_ent = T // m
+        self.codes = np.empty((n_ent, 256), np.uint8)
+        self.scales = np.empty((n_ent, 32), np.uint8)
+        self.keys8 = np.empty((n_ent, 128), np.uint8)
+        step = 65536
+        for t0 in range(0, n_ent * m, step):
+            t1 = min(n_ent * m, t0 + step)
+            lat, key, gate = synth.tokens(w, b, t0, t1, "cpu", chan)
+            c, s, k = oracle.build_entries(m, lat.numpy(), key.numpy(), gate.numpy())
+            self.codes[t0 // m: t1 // m], self.scales[t0 // m: t1 // m], self.keys8[t0 // m: t1 // m] = c, s, k
+        self.summ = oracle.build_summaries(self.keys8)
+        nv = min(T, 128)
+        tail, _, _ = synth.tokens(w, b, T - nv, T, "cpu", chan)
+        wc, ws, _ = oracle.swa_window(tail.numpy(), T)
+        self.win = (wc[:nv], ws[:nv])
+        self.layers = []
+        for li in range(len(w.layers)):
+            q, qi, hw = synth.queries(w, li)
+            self.layers.append((q[b].view(torch.int16).numpy().view(np.uint16),
+                                qi[b].view(torch.int16).numpy().view(np.uint16), hw[b].numpy()))
+        self.units = self._units()
+
+    def _units(self):
+        """List of callables; running all of them in order is one full step."""
+        w, o = self.w, self.o
+        st = {}
+        units = []
+        nb = self.summ.shape[0]
+        n_ent = self.keys8.shape[0]
+        for li, mode in enumerate(w.layers):
+            q, qi, hw = self.layers[li]
+            if mode == "full" and w.index == "flat":
+                st_scores = np.empty(n_ent, np.float32)
+                for c0 in range(0, n_ent, self.CHUNK):
+                    units.append(lambda c0=c0, qi=qi, hw=hw, s=st_scores:
+                                 s.__setitem__(slice(c0, c0 + self.CHUNK),
+                                               o.score_f32(qi, hw, self.keys8[c0:c0 + self.CHUNK])))
+                units.append(lambda s=st_scores: st.__setitem__("top", o.topk(s, 512)))
+            elif mode == "full":
+                bsc = np.empty(nb, np.float32)
+                for c0 in range(0, nb, self.CHUNK):
+                    units.append(lambda c0=c0, qi=qi, hw=hw, s=bsc:
+                                 s.__setitem__(slice(c0, c0 + self.CHUNK),
+                                               o.score_f32(qi, hw, self.summ[c0:c0 + self.CHUNK])))
+
+                def pool_unit(s=bsc):
+                    blocks = o.topk(s, 2048)
+                    st["pool"], st["plen"] = o.expand_pool(blocks, n_ent)
+                units.append(pool_unit)
+                units.append(lambda qi=qi, hw=hw: st.__setitem__(
+                    "top", o.index_pool(qi, hw, self.keys8, st["pool"], st["plen"])))
+            elif mode == "reindex":
+                units.append(lambda qi=qi, hw=hw: st.__setitem__(
+                    "top", o.index_pool(qi, hw, self.keys8, st["pool"], st["plen"])))
+
+            def attend_unit(q=q):
+                ids = st["top"][st["top"] >= 0]
+                st["out"] = o.attend(q, self.codes[ids], self.scales[ids], self.win[0], self.win[1],
+                                     1.0 / math.sqrt(512.0))
+            units.append(attend_unit)
+        return units
+
+    def run_full(self):
+        for u in self.units:
+            u()
+
+
+def cpu_baseline(w: synth.Workload, repeats: int = 4) -> dict:
+    q = OracleQuery(w, 0)
+    q.run_full()
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        q.run_full()
+    dt = time.perf_counter() - t0
+    return {"value": repeats / dt, "unit": "queries/s", "cores": 1, "kind": "oracle",
+            "sample": f"{repeats} x one request's full step ({w.name}, request 0, {len(q.units)} stages), "
+                      f"single-threaded C oracle"}
+
+
+def run_reference(args, w: synth.Workload, rank: int, world: int):
+    if rank != 0:
+        return
+    q = OracleQuery(w, 0)
+    U = len(q.units)
+    k = 0
+    for _ in range(args.warmup):
+        q.units[k % U]()
+        k += 1
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        q.units[k % U]()
+        k += 1
+    dt = time.perf_counter() - t0
+    value = (args.steps / U) / dt
+    line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": 1, "sample": "one request, stage units round-robin"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step = one of the {U} stage units of one request's decode step "
+                                       f"(round-robin; {U} steps = one query)"},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU side
+def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
+    import csa2_sparse_attention_decode_b200 as csa2
+    from csa2_sparse_attention_decode_b200.harness import DeviceWorkload
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dw = DeviceWorkload(w, dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    dom_kernel = csa2.KERNEL_FLAT_SCORE if w.index == "flat" else csa2.KERNEL_BLOCK_SCORE
+    k_start = torch.cuda.Event(enable_timing=True)
+    k_stop = torch.cuda.Event(enable_timing=True)
+
+    # warm up eagerly once (first-call attribute set-up happens outside capture)
+    with torch.cuda.stream(stream):
+        dw.restore(stream)
+        dw.step(stream)
+    stream.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache, stream) == 0
+
+    # torch only reports elapsed time between events it has recorded itself;
+    # record the pair once so later records by the library are readable.
+    k_start.record(stream)
+    k_stop.record(stream)
+    stream.synchronize()
+    csa2.csa2_set_profile_events(dom_kernel, k_start, k_stop)
+    graph = torch.cuda.CUDAGraph()
+    n0 = csa2.csa2_launch_count()
+    with torch.cuda.graph(graph, stream=stream):
+        dw.step(stream)
+    launches_per_step = csa2.csa2_launch_count() - n0
+    csa2.csa2_set_profile_events(dom_kernel, None, None)
+
+    def one(timed_events=None):
+        with torch.cuda.stream(stream):
+            if w.append:
+                dw.restore(stream)
+            flush.zero_()
+            if timed_events:
+                timed_events[0].record(stream)
+            graph.replay()
+            if timed_events:
+                timed_events[1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        one()
+    stream.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    step_ms, kern_ms = [], []
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+    for i in range(args.steps):
+        e = ev[i % 2]
+        one(e)
+        stream.synchronize()
+        step_ms.append(e[0].elapsed_time(e[1]))
+        kern_ms.append(k_start.elapsed_time(k_stop))
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    queries = world * w.batch * args.steps
+    value = queries / (max_total_ms / 1e3)
+
+    # ---- end to end: pinned host inputs -> device, replay, outputs -> host
+    ins = [x for li, mode in enumerate(w.layers) for x in
+           ((dw.layers[li][0],) + ((dw.layers[li][1], dw.layers[li][2]) if mode != "reuse" else ()))]
+    if w.append:
+        ins += list(dw.new)
+    host_in = [x.detach().cpu().pin_memory() for x in ins]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in dw.outs]
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    e2e_steps = max(3, min(args.steps, 200))
+    e2e_ms = []
+    for i in range(e2e_steps + 3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            if w.append:
+                dw.restore(stream)
+            flush.zero_()
+            a.record(stream)
+            for d, h in zip(ins, host_in):
+                d.copy_(h, non_blocking=True)
+            graph.replay()
+            for h, o in zip(host_out, dw.outs):
+                h.copy_(o, non_blocking=True)
+            b.record(stream)
+        stream.synchronize()
+        if i >= 3:
+            e2e_ms.append(a.elapsed_time(b))
+    te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = world * w.batch * e2e_steps / (float(te.item()) / 1e3)
+
+    # ---- roofline of the dominant kernel (live CUDA-event timing)
+    ab = algorithmic_bytes(w)
+    kbytes = ab["block_summaries"] if w.index != "flat" else ab["index"]
+    kern_avg_ms = statistics.mean(kern_ms)
+    achieved = kbytes / (kern_avg_ms / 1e3) / 1e9
+    peak, peak_src = measured_peak_hbm()
+    step_avg_ms = max_total_ms / args.steps
+    roofline = {"bound": "hbm", "kernel": "block_score" if w.index != "flat" else "flat_score",
+                "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel_ms": kern_avg_ms, "kernel_share_of_step": kern_avg_ms / step_avg_ms,
+                "algorithmic_bytes_per_launch": kbytes,
+                "step_achieved_gbs": ab["step"] / (step_avg_ms / 1e3) / 1e9,
+                "step_frac": ab["step"] / (step_avg_ms / 1e3) / 1e9 / peak,
+                "step_algorithmic_bytes": ab["step"]}
+
+    line = None
+    if rank == 0:
+        cpu = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
+        line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": step_avg_ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+                "config": {"workload": w.name, "batch_per_gpu": w.batch, "entries_per_request": w.n_entries[0],
+                           "heads": w.heads, "layers": w.layers, "index": w.index,
+                           "l2": "flushed between timed steps (256 MB write, not timed)",
+                           "timing": "CUDA graph replay of one step, CUDA events per step"},
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": int(launches_per_step * args.steps),
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    del graph
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--small", action="store_true", help="small variant of the workload (testing only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        backend = "nccl" if (torch.cuda.is_available() and args.impl != "reference") else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    w = synth.workload(args.config, small=args.small)
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, rank, world)
+        else:
+            run_gpu(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+// extern "C" entry points of libcsa2: host-side validation, workspace layout
+// and kernel dispatch.  See include/csa2.h for the contract of each call.
+#include <atomic>
+#include <cstdio>
+
+#include "common.cuh"
+#include "index.cuh"
+
+using namespace csa2;
+
+namespace {
+
+std::atomic<unsigned long long> g_launches{0};
+cudaEvent_t g_prof[CSA2_KERNEL_COUNT][2] = {};
+
+}  // namespace
+
+void csa2::note_launch(int kernel, cudaStream_t st, bool before)
+{
+    if (!before) g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (kernel >= 0 && kernel < CSA2_KERNEL_COUNT && g_prof[kernel][before ? 0 : 1])
+        cudaEventRecord(g_prof[kernel][before ? 0 : 1], st);
+}
+
+namespace {
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace layout (all regions 256-byte aligned):
+//   scores_a [batch][row_stride] f32  row scores (entries or blocks)
+//   scores_b [batch][16384]      f32  pool scores
+//   blocks   [batch][2048]       i32  selected blocks (FULL)
+//   part_ml  [batch][10][heads][2] f32, part_o [batch][10][heads][512] f32
+struct Workspace {
+    float *scores_a, *scores_b, *part_ml, *part_o;
+    int32_t *blocks;
+    int64_t row_stride;
+    size_t bytes;
+};
+
+Workspace layout(void *base, int32_t batch, int32_t heads, int32_t max_entries)
+{
+    Workspace w{};
+    w.row_stride = ((int64_t)max_entries + 3) & ~(int64_t)3;
+    size_t off = 0;
+    auto take = [&](size_t n) { size_t o = off; off = align256(off + n); return (char *)base + o; };
+    w.scores_a = (float *)take(sizeof(float) * (size_t)batch * (size_t)w.row_stride);
+    w.scores_b = (float *)take(sizeof(float) * (size_t)batch * CSA2_POOL);
+    w.blocks = (int32_t *)take(sizeof(int32_t) * (size_t)batch * CSA2_MAX_BLOCKS);
+    w.part_ml = (float *)take(sizeof(float) * (size_t)batch * ATT_SPLITS * heads * 2);
+    w.part_o = (float *)take(sizeof(float) * (size_t)batch * ATT_SPLITS * heads * CSA2_LATENT);
+    w.bytes = off;
+    return w;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+csa2_status check_cache(const csa2_cache *c)
+{
+    if (!c || !c->pool || !c->page_table || !c->n_tokens || !c->m || !c->swa || !c->pending || !c->error)
+        return CSA2_ERR_INVALID_ARG;
+    if (c->batch <= 0 || c->n_pages <= 0 || c->max_pages <= 0) return CSA2_ERR_INVALID_ARG;
+    if ((int64_t)c->max_pages * CSA2_PAGE_ENTRIES > (int64_t)1 << 30) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(c->pool, 256) || !aligned(c->swa, 256) || !aligned(c->pending, 16)) return CSA2_ERR_INVALID_ARG;
+    return CSA2_OK;
+}
+
+csa2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t csa2_page_bytes(void) { return CSA2_PAGE_BYTES; }
+size_t csa2_swa_bytes(void) { return CSA2_SWA_BYTES; }
+
+size_t csa2_workspace_bytes(int32_t batch, int32_t heads, int32_t max_entries)
+{
+    if (batch <= 0 || heads <= 0 || max_entries < 0) return 0;
+    return layout(nullptr, batch, heads, max_entries).bytes;
+}
+
+csa2_status csa2_prefill(const csa2_cache *cache, int32_t req, int32_t m_host, int32_t tok_begin, int32_t n_tok,
+                         int32_t n_tok_final, const float *lat, const float *key, const float *gate,
+                         csa2_stream_t stream)
+{
+    csa2_status st = check_cache(cache);
+    if (st != CSA2_OK) return st;
+    if (req < 0 || req >= cache->batch || (m_host != 1 && m_host != 2)) return CSA2_ERR_INVALID_ARG;
+    if (tok_begin < 0 || n_tok < 0 || tok_begin % m_host != 0 || tok_begin + n_tok > n_tok_final)
+        return CSA2_ERR_INVALID_ARG;
+    if ((int64_t)(tok_begin + n_tok) / m_host > (int64_t)cache->max_pages * CSA2_PAGE_ENTRIES)
+        return CSA2_ERR_INVALID_ARG;
+    if (n_tok > 0 && (!lat || !key || !gate)) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(lat, 16) || !aligned(key, 16)) return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_prefill(make_view(cache), req, m_host, tok_begin, n_tok, n_tok_final, lat, key, gate,
+                                    (cudaStream_t)stream));
+}
+
+csa2_status csa2_append(const csa2_cache *cache, const float *lat, const float *key, const float *gate,
+                        const int32_t *n_new, csa2_stream_t stream)
+{
+    csa2_status st = check_cache(cache);
+    if (st != CSA2_OK) return st;
+    if (!lat || !key || !gate || !n_new) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(lat, 16) || !aligned(key, 16)) return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_append(make_view(cache), lat, key, gate, n_new, (cudaStream_t)stream));
+}
+
+csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint16_t *q_idx, const float *w,
+                       int32_t *pool, int32_t *pool_len, int32_t *topk, void *ws, size_t ws_bytes,
+                       csa2_stream_t stream)
+{
+    csa2_status st = check_cache(cache);
+    if (st != CSA2_OK) return st;
+    if (!q_idx || !w || !topk || !ws || !aligned(ws, 256)) return CSA2_ERR_INVALID_ARG;
+    if (mode != CSA2_INDEX_FLAT && mode != CSA2_INDEX_FULL && mode != CSA2_INDEX_REINDEX) return CSA2_ERR_INVALID_ARG;
+    if (mode != CSA2_INDEX_FLAT && (!pool || !pool_len)) return CSA2_ERR_INVALID_ARG;
+    const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
+    Workspace W = layout(ws, cache->batch, 1, max_entries);
+    if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
+    CacheView c = make_view(cache);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (mode == CSA2_INDEX_FLAT) {
+        e = launch_score(c, ROWS_KEYS, q_idx, w, nullptr, nullptr, W.scores_a, W.row_stride, max_entries, s);
+        if (e == cudaSuccess)
+            e = launch_select(c, ROWS_KEYS, W.scores_a, W.row_stride, nullptr, nullptr, CSA2_TOPK, topk, CSA2_TOPK,
+                              0, nullptr, nullptr, s);
+        return from_cuda(e);
+    }
+    if (mode == CSA2_INDEX_FULL) {
+        const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
+        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores_a, W.row_stride, max_blocks, s);
+        if (e == cudaSuccess)
+            e = launch_select(c, ROWS_SUMMARIES, W.scores_a, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS,
+                              W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, s);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    e = launch_score(c, ROWS_POOL, q_idx, w, pool, pool_len, W.scores_b, CSA2_POOL, CSA2_POOL, s);
+    if (e == cudaSuccess)
+        e = launch_select(c, ROWS_POOL, W.scores_b, CSA2_POOL, pool_len, pool, CSA2_TOPK, topk, CSA2_TOPK, 0,
+                          nullptr, nullptr, s);
+    return from_cuda(e);
+}
+
+csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *q, const int32_t *topk, float scale,
+                        void *out, int32_t out_is_fp32, void *ws, size_t ws_bytes, csa2_stream_t stream)
+{
+    csa2_status st = check_cache(cache);
+    if (st != CSA2_OK) return st;
+    if (heads <= 0 || heads > 128 || !q || !topk || !out || !ws || !aligned(ws, 256)) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(out, 16)) return CSA2_ERR_INVALID_ARG;
+    const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
+    Workspace W = layout(ws, cache->batch, heads, max_entries);
+    if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, W.part_o, W.part_ml,
+                                   (cudaStream_t)stream));
+}
+
+csa2_status csa2_get_device_error(const csa2_cache *cache, int32_t *code_out, csa2_stream_t stream)
+{
+    if (!cache || !cache->error || !code_out) return CSA2_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, cache->error, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(cache->error, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    *code_out = v;
+    return v == 0 ? CSA2_OK : CSA2_ERR_DEVICE_CHECK;
+}
+
+csa2_status csa2_set_profile_events(int32_t kernel, void *ev_start, void *ev_stop)
+{
+    if (kernel < 0 || kernel >= CSA2_KERNEL_COUNT || (!ev_start) != (!ev_stop)) return CSA2_ERR_INVALID_ARG;
+    g_prof[kernel][0] = (cudaEvent_t)ev_start;
+    g_prof[kernel][1] = (cudaEvent_t)ev_stop;
+    return CSA2_OK;
+}
+
+uint64_t csa2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *csa2_status_string(csa2_status status)
+{
+    switch (status) {
+    case CSA2_OK: return "ok";
+    case CSA2_ERR_INVALID_ARG: return "invalid argument";
+    case CSA2_ERR_UNSUPPORTED: return "unsupported";
+    case CSA2_ERR_CUDA: return "CUDA error";
+    case CSA2_ERR_DEVICE_CHECK: return "device-side data check failed";
+    case CSA2_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

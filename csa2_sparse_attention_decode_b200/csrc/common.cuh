@@ -1,0 +1,131 @@
+// Device-side helpers shared by the libcsa2 kernels: number formats, page
+// addressing and the device error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+// ---------------------------------------------------------------- diagnostics
+// Defined in capi.cu: launch counting and optional event brackets.
+void note_launch(int kernel, cudaStream_t st, bool before);
+
+struct LaunchScope {
+    int k;
+    cudaStream_t st;
+    LaunchScope(int kernel, cudaStream_t s) : k(kernel), st(s) { note_launch(k, st, true); }
+    ~LaunchScope() { note_launch(k, st, false); }
+};
+
+// ---------------------------------------------------------------- errors
+__device__ __forceinline__ void set_error(int32_t *err, int32_t code)
+{
+    if (err) atomicCAS(err, 0, code);
+}
+
+// ---------------------------------------------------------------- formats
+// e4m3 with round-to-nearest-even and saturation to +-448 (the fp8 KV /
+// indexer-key format of the CSA2 config).
+__device__ __forceinline__ uint8_t f32_to_e4m3(float x)
+{
+    return (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c)
+{
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+// e2m1 magnitude code of a = |x| with round-to-nearest, ties to the even code
+// (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; saturating).  Ties sit at the
+// midpoints .25 .75 1.25 1.75 2.5 3.5 5: a tie goes up exactly when the upper
+// neighbour has the even code.
+__device__ __forceinline__ uint32_t e2m1_mag_code(float a)
+{
+    return (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+           (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
+           (uint32_t)(a > 5.0f);
+}
+
+__device__ __forceinline__ uint32_t f32_to_e2m1(float x)
+{
+    uint32_t sign = (__float_as_uint(x) >> 31) << 3;
+    return sign | e2m1_mag_code(fabsf(x));
+}
+
+// Smallest integer e with amax <= 448 * 2^e (amax > 0, finite).
+__device__ __forceinline__ int swa_exponent(float amax)
+{
+    int ex;
+    float f = frexpf(amax, &ex);          // amax = f * 2^ex, f in [0.5, 1)
+    return (f > 0.875f) ? ex - 8 : ex - 9;
+}
+
+// ---------------------------------------------------------------- layout
+struct CacheView {
+    uint8_t *pool;
+    int32_t n_pages;
+    const int32_t *page_table;
+    int32_t max_pages;
+    int32_t *n_tokens;
+    const int32_t *m;
+    uint8_t *swa;
+    float *pending;
+    int32_t *error;
+    int32_t batch;
+};
+
+__host__ inline CacheView make_view(const csa2_cache *c)
+{
+    CacheView v;
+    v.pool = (uint8_t *)c->pool;
+    v.n_pages = c->n_pages;
+    v.page_table = c->page_table;
+    v.max_pages = c->max_pages;
+    v.n_tokens = c->n_tokens;
+    v.m = c->m;
+    v.swa = (uint8_t *)c->swa;
+    v.pending = c->pending;
+    v.error = c->error;
+    v.batch = c->batch;
+    return v;
+}
+
+// Page base of entry e (or block e/8) of request b; nullptr (and the error
+// word set) when the page slot or page id is out of range.
+__device__ __forceinline__ uint8_t *entry_page(const CacheView &c, int b, int e)
+{
+    int pi = e >> 6;
+    if (e < 0 || pi >= c.max_pages) {
+        set_error(c.error, CSA2_DEV_CAPACITY);
+        return nullptr;
+    }
+    int pid = __ldg(c.page_table + (size_t)b * c.max_pages + pi);
+    if (pid < 0 || pid >= c.n_pages) {
+        set_error(c.error, CSA2_DEV_BAD_PAGE);
+        return nullptr;
+    }
+    return c.pool + (size_t)pid * CSA2_PAGE_BYTES;
+}
+
+__device__ __forceinline__ uint8_t *swa_base(const CacheView &c, int b)
+{
+    return c.swa + (size_t)b * CSA2_SWA_BYTES;
+}
+
+// Entries of request b, clamped to the pages it owns (a corrupt n_tokens
+// can never push an index past the request's capacity).
+__device__ __forceinline__ int n_entries_of(const CacheView &c, int b)
+{
+    int m = c.m[b];
+    int n = c.n_tokens[b] / (m == 2 ? 2 : 1);
+    return max(0, min(n, c.max_pages * CSA2_PAGE_ENTRIES));
+}
+
+}  // namespace csa2

@@ -1,0 +1,22 @@
+// Launch entry points of the indexer kernels (host side).
+#pragma once
+#include "common.cuh"
+
+namespace csa2 {
+enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2 };
+
+cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,
+                         const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st);
+cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
+                          const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
+                          int32_t *pool_len, cudaStream_t st);
+cudaError_t launch_prefill(const CacheView &c, int req, int m, int tok_begin, int n_tok, int n_tok_final,
+                           const float *lat, const float *key, const float *gate, cudaStream_t st);
+cudaError_t launch_append(const CacheView &c, const float *lat, const float *key, const float *gate,
+                          const int32_t *n_new, cudaStream_t st);
+cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
+                          void *out, int out_is_fp32, float *part_o, float *part_ml, cudaStream_t st);
+
+constexpr int ATT_KEYS_PER_SPLIT = 64;
+constexpr int ATT_SPLITS = (CSA2_TOPK + CSA2_SWA) / ATT_KEYS_PER_SPLIT;   // 10
+}  // namespace csa2

@@ -1,0 +1,227 @@
+/*
+ * csa2.h -- C ABI of libcsa2, the B200 (sm_100a) CSA2 sparse-attention
+ * decode step over a compressed, FP4-quantised global KV cache.
+ *
+ * The method (DeepSeek-V4.1-Flash CSA2) is described by:
+ *   [blog-0539] 0539edu.com/news/5732216, §1 (each m tokens become one cache
+ *               entry; main KV, indexer K and top-k indices are reused across
+ *               layers) and §3 (layer modes Full / Reuse / Reindex; the
+ *               config: fp4_e2m1 global KV with one e4m3 scale per 16
+ *               channels, fp8 SWA KV with a 128-token window, indexer of
+ *               32 heads x 128 dims with top_k 512, hierarchical selection of
+ *               2048 blocks x 8 positions = a 16384-candidate pool; the Full
+ *               layer builds the pool and Reindex layers search inside it).
+ *   [daiw]      daiw.net/manual/deepseek-v4-flash/million-token-cost: decode
+ *               reads the cache every step and is bandwidth-bound; the
+ *               cache-size factor table (one 512-dim KV shared by all query
+ *               heads).
+ *   [nxbn]      m.nxbn.cn/news/78290 §3.1 (E2M1 = 2 exponent bits, 1 mantissa
+ *               bit), §4.2 (gated weighted compression of m tokens).
+ *
+ * Conventions shared by every call:
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or synchronises, except csa2_get_device_error,
+ *     which synchronises the given stream.
+ *   - Every call enqueues asynchronously on `stream` (0 = legacy default).
+ *   - The return value reports host-side argument validation
+ *     (CSA2_ERR_INVALID_ARG, nothing enqueued) and launch errors
+ *     (CSA2_ERR_CUDA).  Errors found in the DATA on the device (a page id
+ *     outside the pool, an entry index beyond a request's pages, a top-k index
+ *     beyond the request's entries, a bad m or n_new) never trap: the kernel
+ *     skips that element and records the first such code in cache->error;
+ *     read it with csa2_get_device_error.
+ *   - Multi-byte values are little-endian; bf16 values are passed as their
+ *     16-bit patterns (uint16_t).
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csa2_stream_t;   /* == cudaStream_t */
+
+/* ---- method constants ([blog-0539] §3 config) ------------------------- */
+#define CSA2_LATENT        512    /* shared latent (K = V) dim ([daiw])         */
+#define CSA2_SCALE_GROUP   16     /* channels per e4m3 scale                    */
+#define CSA2_CODE_BYTES    256    /* FP4 codes per entry: 512 x 4 bit           */
+#define CSA2_SCALE_BYTES   32     /* e4m3 scales per entry: 512 / 16            */
+#define CSA2_KEY_DIM       128    /* indexer head_dim; FP8 key bytes per entry  */
+#define CSA2_IDX_HEADS     32     /* indexer query_heads                        */
+#define CSA2_BLOCK         8      /* positions_per_block                        */
+#define CSA2_MAX_BLOCKS    2048   /* max_blocks                                 */
+#define CSA2_POOL          16384  /* candidate_pool_size = 2048 x 8             */
+#define CSA2_TOPK          512    /* top_k                                      */
+#define CSA2_SWA           128    /* swa_window_size                            */
+
+/* ---- cache layout -------------------------------------------------------
+ * Global KV lives in one pool of fixed-size pages of 64 entries.  Entry e of
+ * request b lives in page page_table[b * max_pages + (e >> 6)], slot e & 63.
+ * Inside a page the fields are stored as separate arrays (each 256-byte
+ * aligned within the page):
+ *   codes     [64][256] u8   FP4 e2m1 codes; byte j = channel 2j (low nibble)
+ *                            | channel 2j+1 (high nibble); bit 3 = sign
+ *   scales    [64][32]  u8   e4m3 scale of channels 16i .. 16i+15
+ *   keys      [64][128] u8   FP8 e4m3 indexer key
+ *   summaries [8][128]  u8   FP8 e4m3 mean of the keys of block (e >> 3)
+ * Per request, the SWA ring holds the last min(n_tokens, 128) raw tokens:
+ *   codes [128][512] u8 e4m3, then scale [128] f32 (a power of two); token
+ *   position t sits in slot t % 128.                                         */
+#define CSA2_PAGE_ENTRIES      64
+#define CSA2_PAGE_CODES_OFF    0
+#define CSA2_PAGE_SCALES_OFF   16384
+#define CSA2_PAGE_KEYS_OFF     18432
+#define CSA2_PAGE_SUMM_OFF     26624
+#define CSA2_PAGE_BYTES        27648
+#define CSA2_SWA_CODES_OFF     0
+#define CSA2_SWA_SCALE_OFF     65536
+#define CSA2_SWA_BYTES         66048
+#define CSA2_PENDING_STRIDE    656    /* floats: latent 512 | key 128 | gate 1 | pad */
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,
+    CSA2_ERR_UNSUPPORTED = 2,
+    CSA2_ERR_CUDA = 3,
+    CSA2_ERR_DEVICE_CHECK = 4,
+    CSA2_ERR_TIMEOUT = 5
+} csa2_status;
+
+/* Device error word values (cache->error). */
+#define CSA2_DEV_OK              0
+#define CSA2_DEV_BAD_PAGE        1   /* page id outside [0, n_pages)            */
+#define CSA2_DEV_CAPACITY        2   /* entry index >= max_pages * 64           */
+#define CSA2_DEV_BAD_INDEX       3   /* top-k / pool index outside the request  */
+#define CSA2_DEV_BAD_REQUEST     4   /* m not in {1,2}, n_new not in [0,2], ... */
+
+typedef enum {
+    CSA2_INDEX_FLAT = 0,     /* exact top-512 over every entry                   */
+    CSA2_INDEX_FULL = 1,     /* hierarchical: blocks -> pool -> top-512; writes pool */
+    CSA2_INDEX_REINDEX = 2   /* rescore a given pool, top-512                    */
+} csa2_index_mode;
+
+/* A batch of requests' caches.  The struct itself is host memory and is read
+ * only during the call; every pointer in it is a device pointer owned by the
+ * caller and must stay valid until the enqueued work completes. */
+typedef struct {
+    void          *pool;        /* n_pages * CSA2_PAGE_BYTES, 256-byte aligned          */
+    int32_t        n_pages;
+    const int32_t *page_table;  /* [batch][max_pages]                                   */
+    int32_t        max_pages;   /* pages per request; entry capacity = 64 * max_pages   */
+    int32_t       *n_tokens;    /* [batch] tokens seen; entries = n_tokens / m          */
+    const int32_t *m;           /* [batch] compression ratio, 1 or 2                    */
+    void          *swa;         /* [batch] * CSA2_SWA_BYTES, 256-byte aligned           */
+    float         *pending;     /* [batch][CSA2_PENDING_STRIDE]: an m=2 request's odd token */
+    int32_t       *error;       /* one device word; 0 = no data error                   */
+    int32_t        batch;
+} csa2_cache;
+
+/* Sizes ------------------------------------------------------------------ */
+size_t csa2_page_bytes(void);   /* CSA2_PAGE_BYTES */
+size_t csa2_swa_bytes(void);    /* CSA2_SWA_BYTES  */
+
+/* Bytes of workspace csa2_index and csa2_attend need for `batch` requests of
+ * at most `max_entries` entries with `heads` attention heads.  The caller
+ * allocates it (256-byte aligned) and may share one workspace between calls
+ * that run in stream order. */
+size_t csa2_workspace_bytes(int32_t batch, int32_t heads, int32_t max_entries);
+
+/* Bulk build (prefill side) ----------------------------------------------
+ * Compress and pack tokens [tok_begin, tok_begin + n_tok) of request `req`
+ * ([blog-0539] §1: m tokens -> one entry; [nxbn] §4.2: entry = sum_i
+ * softmax(g)_i x_i over the m tokens of a group, for the latent and the
+ * indexer key alike; m = 1 copies).  Writes the FP4 codes + e4m3 scales,
+ * the FP8 key, recomputes the summaries of every block it touches, writes
+ * tokens at positions >= n_tok_final - 128 into the SWA ring, keeps an m=2
+ * request's unpaired last token in `pending`, and sets
+ * n_tokens[req] = tok_begin + n_tok.
+ *   lat  [n_tok][512] f32, key [n_tok][128] f32, gate [n_tok] f32 (device).
+ *   tok_begin must be a multiple of m (read from m_host, which must equal
+ *   cache->m[req]); calls for one request go in increasing tok_begin. */
+csa2_status csa2_prefill(const csa2_cache *cache, int32_t req, int32_t m_host,
+                         int32_t tok_begin, int32_t n_tok, int32_t n_tok_final,
+                         const float *lat, const float *key, const float *gate,
+                         csa2_stream_t stream);
+
+/* Decode-step append ([blog-0539] §1, §3; [nxbn] §4.2) -------------------
+ * Request b appends n_new[b] in {0,1,2} raw tokens: lat [batch][2][512],
+ * key [batch][2][128], gate [batch][2] (f32, rows past n_new ignored).
+ * Every new token enters the SWA ring as FP8 with a per-token power-of-two
+ * scale; m=1 turns each token into an entry; m=2 pairs the pending odd token
+ * (if any) with the new ones, completing entries and keeping a leftover
+ * token pending.  Each new entry is packed as FP4 e2m1 + e4m3 per-16 scales
+ * with its key in FP8, the summary of its block is recomputed, and
+ * n_tokens[b] += n_new[b]. */
+csa2_status csa2_append(const csa2_cache *cache, const float *lat, const float *key,
+                        const float *gate, const int32_t *n_new, csa2_stream_t stream);
+
+/* Indexer ([blog-0539] §3 indexer and hierarchical blocks, and the passage
+ * that follows: Full builds the pool, Reindex searches only inside it) ----
+ * score(row) = sum_h w_h * ReLU(q_idx_h . row) with q_idx bf16 [batch][32][128]
+ * and w f32 [batch][32], rows being FP8 keys or block summaries.
+ *   FLAT:    top-min(512, N) entries of all N.
+ *   FULL:    top-min(2048, ceil(N/8)) blocks by summary score; their entries
+ *            (ascending) form pool[b][0 .. pool_len[b]) (rest -1); exact
+ *            rescoring of the pool's keys; top-min(512, pool_len).
+ *   REINDEX: the pool/pool_len given (as written by a FULL call) is
+ *            rescored with this layer's q_idx/w; top-min(512, pool_len).
+ * topk[b][512] receives entry indices in ascending order, -1 padded.  Order
+ * of selection: score descending, ties to the lower index.  pool and
+ * pool_len are [batch][16384] / [batch] int32; unused (may be NULL) in FLAT
+ * mode.  ws / ws_bytes: workspace of at least csa2_workspace_bytes(). */
+csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode,
+                       const uint16_t *q_idx, const float *w,
+                       int32_t *pool, int32_t *pool_len, int32_t *topk,
+                       void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* Sparse MQA decode attention ([daiw] decode step and factor table: one
+ * 512-dim latent shared by all heads, used as both K and V) --------------
+ * For every head h of request b:
+ *   o_h = sum_j softmax_j(scale * q_h . v_j) v_j
+ * over j in {valid topk[b][*] entries (FP4 e2m1 x e4m3 scale)} plus the
+ * min(n_tokens[b], 128) SWA tokens (FP8 x power-of-two scale), one softmax,
+ * no de-duplication.  q bf16 [batch][heads][512]; heads in 1..128.
+ * out [batch][heads][512] is bf16 (out_is_fp32 = 0) or f32 (= 1).  A request
+ * with no keys gets a zero output.  Reuse layers call this with their
+ * group's topk and their own q. */
+csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *q,
+                        const int32_t *topk, float scale, void *out, int32_t out_is_fp32,
+                        void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* Diagnostics ------------------------------------------------------------
+ * Kernels that csa2_set_profile_events can bracket with CUDA events. */
+typedef enum {
+    CSA2_KERNEL_BLOCK_SCORE = 0,   /* FULL: scoring of the block summaries     */
+    CSA2_KERNEL_FLAT_SCORE = 1,    /* FLAT: scoring of every key               */
+    CSA2_KERNEL_POOL_SCORE = 2,    /* FULL / REINDEX: exact pool rescoring     */
+    CSA2_KERNEL_SELECT = 3,        /* radix top-k                              */
+    CSA2_KERNEL_ATTEND = 4,        /* split-KV attention partials              */
+    CSA2_KERNEL_COMBINE = 5,       /* log-sum-exp combine                      */
+    CSA2_KERNEL_COUNT = 6
+} csa2_kernel_id;
+
+/* When ev_start / ev_stop (cudaEvent_t, created by the caller with timing
+ * enabled) are non-NULL, every later launch of `kernel` is preceded by
+ * cudaEventRecord(ev_start) and followed by cudaEventRecord(ev_stop) on the
+ * stream it is launched on, so the pair brackets the most recent launch.
+ * Pass NULLs to stop.  Process-wide setting; not thread-safe. */
+csa2_status csa2_set_profile_events(int32_t kernel, void *ev_start, void *ev_stop);
+
+/* Number of kernels this library has launched in this process so far. */
+uint64_t csa2_launch_count(void);
+
+/* Synchronises `stream`, copies cache->error into *code_out and resets the
+ * device word to 0. */
+csa2_status csa2_get_device_error(const csa2_cache *cache, int32_t *code_out,
+                                  csa2_stream_t stream);
+
+const char *csa2_status_string(csa2_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

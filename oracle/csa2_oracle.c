@@ -233,7 +233,8 @@ void orc_build_entries(int m, int e_begin, int e_end,
     for (int e = e_begin; e < e_end; ++e) {
         int r = (e - e_begin) * m;
         for (int i = 0; i < m; ++i) {
-            memcpy(lat + i * OR_LATENT, tok_lat + (size_t)(r + i) * OR_LATENT, sizeof(float) * OR_LATENT);
+            if (codes || scales)
+                memcpy(lat + i * OR_LATENT, tok_lat + (size_t)(r + i) * OR_LATENT, sizeof(float) * OR_LATENT);
             memcpy(key + i * OR_IDX_DIM, tok_key + (size_t)(r + i) * OR_IDX_DIM, sizeof(float) * OR_IDX_DIM);
         }
         const float *g = tok_gate + r;

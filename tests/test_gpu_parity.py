@@ -1,0 +1,244 @@
+"""GPU path vs the oracle, element by element, on seeded synthetic inputs,
+through the C ABI.  Bit-exact for packed bytes and index sets (up to allowed
+boundary swaps), within 2e-3 abs + 1e-3 rel for attention."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import OracleRequest, bits, check_attention, check_swaps
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import csa2_sparse_attention_decode_b200 as csa2
+    from csa2_sparse_attention_decode_b200.harness import SOFTMAX_SCALE, DeviceWorkload
+
+
+def _tiny_workload(n_tok, m, batch=1):
+    return synth.Workload("tiny", 99, batch, 16, [n_tok] * batch, [m] * batch, "flat", ["full"], False,
+                          outliers=False)
+
+
+# ------------------------------------------------------------------ formats / packing
+@pytest.mark.parametrize("m", [1, 2])
+def test_prefill_packs_bit_exact_on_crafted_values(m):
+    gold = __import__("json").load(open(__import__("os").path.join(__import__("os").path.dirname(__file__),
+                                                                   "golden", "fp4_pack_examples.json")))
+    n_tok = 700 * m + (1 if m == 2 else 0)
+    w = _tiny_workload(n_tok, m)
+    dw = DeviceWorkload(w, build=False)
+    g = torch.Generator().manual_seed(5)
+    lat = torch.randn(n_tok, 512, generator=g) * torch.exp(2 * torch.randn(n_tok, 1, generator=g))
+    # crafted groups: the worked examples, ties, zeros, -0, huge (scale saturates), tiny
+    for i, grp in enumerate(gold["groups"]):
+        lat[i, 16:32] = torch.tensor(grp["x"])
+    ties = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5.0, -6.0])
+    lat[5, 0:16] = ties
+    lat[6, :] = 0.0
+    lat[7, :] = -0.0
+    lat[8, :] = 1e5 * torch.randn(512, generator=g)
+    lat[9, :] = 1e-6 * torch.randn(512, generator=g)
+    key = torch.randn(n_tok, 128, generator=g) * 40
+    key[3] = torch.tensor([(c // 2) * 2 ** -9 for c in range(128)])      # subnormal e4m3 ties
+    key[4] = 1000.0
+    gate = torch.randn(n_tok, generator=g) * 3
+    gate[20:24] = torch.tensor([50.0, -50.0, 0.5, 0.5])
+    dev = dw.device
+    for t0 in range(0, n_tok, 256 * m):
+        t1 = min(n_tok, t0 + 256 * m)
+        csa2.csa2_prefill(dw.cache, 0, t0, n_tok, lat[t0:t1].to(dev).contiguous(), key[t0:t1].to(dev).contiguous(),
+                          gate[t0:t1].to(dev).contiguous())
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    N = n_tok // m
+    codes, scales, keys8 = oracle.build_entries(m, lat[:N * m].numpy(), key[:N * m].numpy(), gate[:N * m].numpy())
+    gc, gs, gk = dw.entry_rows(0, torch.arange(N))
+    assert np.array_equal(gc.numpy(), codes)
+    assert np.array_equal(gs.numpy(), scales)
+    assert np.array_equal(gk.numpy(), keys8)
+    summ = oracle.build_summaries(keys8)
+    assert np.array_equal(dw.summary_rows(0, torch.arange(summ.shape[0])).numpy(), summ)
+    sc, ss = dw.swa_rows(0)
+    oc, os_, nv = oracle.swa_window(lat[n_tok - 128:n_tok].numpy(), n_tok)
+    assert np.array_equal(sc.numpy(), oc) and np.array_equal(ss.numpy(), os_)
+    assert int(dw.cache.n_tokens[0]) == n_tok
+    if m == 2:
+        pend = dw.cache.pending[:641].cpu()
+        assert torch.equal(pend[:512], lat[n_tok - 1]) and torch.equal(pend[512:640], key[n_tok - 1])
+
+
+@pytest.mark.parametrize("cid", [0, 2, 4])
+def test_prefill_matches_oracle(cid):
+    w = synth.workload(cid, small=True)
+    dw = DeviceWorkload(w)
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    for b in range(w.batch):
+        ref = OracleRequest(w, b, w.n_tok[b])
+        gc, gs, gk = dw.entry_rows(b, torch.arange(ref.n_entries))
+        assert np.array_equal(gc.numpy(), ref.codes), b
+        assert np.array_equal(gs.numpy(), ref.scales), b
+        assert np.array_equal(gk.numpy(), ref.keys8), b
+        assert np.array_equal(dw.summary_rows(b, torch.arange(ref.summ.shape[0])).numpy(), ref.summ), b
+        sc, ss = dw.swa_rows(b)
+        assert np.array_equal(sc.numpy(), ref.swa_codes) and np.array_equal(ss.numpy(), ref.swa_scale), b
+
+
+@pytest.mark.parametrize("cid", [2, 4])
+def test_append_matches_oracle(cid):
+    w = synth.workload(cid, small=True)
+    dw = DeviceWorkload(w)
+    lat, key, gate, n_new = dw.new
+    csa2.csa2_append(dw.cache, lat, key, gate, n_new)
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    for b in range(w.batch):
+        T = w.n_tok[b] + w.n_new[b]
+        assert int(dw.cache.n_tokens[b]) == T
+        ref = OracleRequest(w, b, T)
+        lo = max(0, w.n_tok[b] // w.m[b] - 9)
+        ids = torch.arange(lo, ref.n_entries)
+        gc, gs, gk = dw.entry_rows(b, ids)
+        assert np.array_equal(gc.numpy(), ref.codes[lo:]), b
+        assert np.array_equal(gs.numpy(), ref.scales[lo:]), b
+        assert np.array_equal(gk.numpy(), ref.keys8[lo:]), b
+        nb = ref.summ.shape[0]
+        assert np.array_equal(dw.summary_rows(b, torch.arange(nb - 2, nb)).numpy(), ref.summ[nb - 2:]), b
+        sc, ss = dw.swa_rows(b)
+        assert np.array_equal(sc.numpy(), ref.swa_codes) and np.array_equal(ss.numpy(), ref.swa_scale), b
+        if w.m[b] == 2 and T % 2 == 1:
+            pend = dw.cache.pending[b * 656: b * 656 + 512].cpu().numpy()
+            assert np.array_equal(pend, ref.lat[T - 1]), b
+
+
+# ------------------------------------------------------------------ index + attend, end to end
+def _check_step(w, dw, refs, check_needles=False):
+    dw.step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    swaps = 0
+    for b in range(w.batch):
+        ref = refs[b]
+        pool = dw.pool[b].cpu().numpy()
+        plen = int(dw.pool_len[b])
+        group_topk = {}
+        for li, mode in enumerate(w.layers):
+            q, q_idx, hw = dw.layers[li]
+            qb, wb = bits(q_idx[b]), hw[b].cpu().numpy()
+            grp = dw.layer_topk[li]
+            gtop = dw.topk[grp][b].cpu().numpy()
+            if mode in ("full", "reindex"):
+                exact = {}
+
+                def score_of(e, qb=qb, wb=wb, exact=exact):
+                    if e not in exact:
+                        exact[e] = float(oracle.score_f64(qb, wb, ref.keys8[e:e + 1])[0])
+                    return exact[e]
+
+                if w.index == "flat":
+                    rtop = oracle.index_flat(qb, wb, ref.keys8)
+                else:
+                    if mode == "full":
+                        # blocks: the GPU pool's block set vs the oracle's block top-k
+                        gblocks = np.unique(pool[:plen] // 8)
+                        bs = oracle.score_f64(qb, wb, ref.summ)
+                        rblocks = oracle.topk(bs.astype(np.float32), 2048)
+                        swaps += check_swaps(gblocks, rblocks, lambda x: bs[x], f"req {b} blocks")
+                        rpool, rplen = oracle.expand_pool(gblocks.astype(np.int32), ref.n_entries)
+                        assert plen == rplen and np.array_equal(pool[:plen], rpool[:rplen]), b
+                    # conditional: the oracle's top-512 inside the GPU's pool
+                    rtop = oracle.index_pool(qb, wb, ref.keys8, pool, plen)
+                swaps += check_swaps(gtop, rtop, score_of, f"req {b} layer {li} top-k")
+                assert np.all(np.diff(gtop[gtop >= 0]) > 0) and (gtop[len(gtop[gtop >= 0]):] == -1).all()
+                if check_needles and mode == "full":
+                    needles = synth.needle_entries(w, b).numpy()
+                    assert set(needles.tolist()) <= set(gtop.tolist()), "needle missed"
+                group_topk[grp] = gtop
+            r = ref.attend(bits(q[b]), gtop, SOFTMAX_SCALE)
+            check_attention(dw.outs[li][b], r, f"req {b} layer {li}")
+    return swaps
+
+
+@pytest.mark.parametrize("cid", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_step_matches_oracle(cid, out_fp32):
+    w = synth.workload(cid, small=True)
+    dw = DeviceWorkload(w, out_fp32=out_fp32)
+    refs = [OracleRequest(w, b, w.n_tok[b] + w.n_new[b]) for b in range(w.batch)]
+    _check_step(w, dw, refs, check_needles=(cid == 1))
+
+
+def test_sharp_softmax_variant():
+    """q ~ N(0,1) (not /sqrt(512)): logits spread enough to exercise the softmax."""
+    w = synth.workload(1, small=True)
+    dw = DeviceWorkload(w, out_fp32=True)
+    q, q_idx, hw = dw.layers[0]
+    dw.layers[0] = ((q.float() * math.sqrt(512)).to(torch.bfloat16), q_idx, hw)
+    refs = [OracleRequest(w, b, w.n_tok[b]) for b in range(w.batch)]
+    _check_step(w, dw, refs)
+
+
+# ------------------------------------------------------------------ invariants
+def test_determinism_and_reuse_of_full_query():
+    w = synth.workload(3, small=True)
+    dw = DeviceWorkload(w)
+    dw.step()
+    a = [o.clone() for o in dw.outs]
+    ta = [t.clone() for t in dw.topk]
+    dw.step()
+    assert all(torch.equal(x, y) for x, y in zip(a, dw.outs))
+    assert all(torch.equal(x, y) for x, y in zip(ta, dw.topk))
+    # a Reuse layer fed the Full layer's own query reproduces its output
+    dw.layers[1] = (dw.layers[0][0], dw.layers[1][1], dw.layers[1][2])
+    dw.step()
+    assert torch.equal(dw.outs[0], dw.outs[1])
+
+
+def test_paging_invariance():
+    w = synth.workload(4, small=True)
+    dw_shuf = DeviceWorkload(w)
+    w_id = synth.workload(4, small=True)
+    w_id.shuffled_pages = False
+    dw_id = DeviceWorkload(w_id)
+    dw_shuf.step()
+    dw_id.step()
+    torch.cuda.synchronize()
+    assert torch.equal(dw_shuf.outs[0], dw_id.outs[0])
+    assert torch.equal(dw_shuf.topk[0], dw_id.topk[0])
+
+
+def test_step_is_repeatable_after_restore():
+    w = synth.workload(4, small=True)
+    dw = DeviceWorkload(w)
+    dw.step()
+    a = dw.outs[0].clone()
+    dw.restore()
+    dw.step()
+    assert torch.equal(a, dw.outs[0])
+
+
+# ------------------------------------------------------------------ device-side data checks
+def test_bad_topk_index_sets_error_and_is_skipped():
+    w = synth.workload(0, small=True)
+    dw = DeviceWorkload(w)
+    dw.step()
+    torch.cuda.synchronize()
+    topk = dw.topk[0].clone()
+    topk[0, 3] = 10 ** 6
+    out = torch.empty_like(dw.outs[0])
+    csa2.csa2_attend(dw.cache, dw.layers[0][0], topk, SOFTMAX_SCALE, out, dw.ws)
+    assert csa2.csa2_get_device_error(dw.cache) == 3
+    assert csa2.csa2_get_device_error(dw.cache) == 0        # read resets the word
+
+
+def test_bad_page_id_sets_error():
+    w = synth.workload(0, small=True)
+    pt = synth.page_table(w)
+    pt[0, 5] = 10 ** 6
+    dw = DeviceWorkload(w, page_table=pt, build=False)
+    lat, key, gate = synth.tokens(w, 0, 0, 2048, "cuda")
+    csa2.csa2_prefill(dw.cache, 0, 0, 2048, lat.contiguous(), key.contiguous(), gate.contiguous())
+    assert csa2.csa2_get_device_error(dw.cache) == 1
