@@ -18,8 +18,17 @@ cudaEvent_t g_prof[CSA2_KERNEL_COUNT][2] = {};
 void csa2::note_launch(int kernel, cudaStream_t st, bool before)
 {
     if (!before) g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (kernel >= 0 && kernel < CSA2_KERNEL_COUNT && g_prof[kernel][before ? 0 : 1])
-        cudaEventRecord(g_prof[kernel][before ? 0 : 1], st);
+    if (kernel < 0 || kernel >= CSA2_KERNEL_COUNT) return;
+    cudaEvent_t ev = g_prof[kernel][before ? 0 : 1];
+    if (!ev) return;
+    // Under stream capture a plain record only marks a dependency; an
+    // external record becomes an event node that fires on every replay.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, st);
 }
 
 namespace {
