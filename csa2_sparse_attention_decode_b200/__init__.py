@@ -26,7 +26,8 @@ INDEX_FLAT, INDEX_FULL, INDEX_REINDEX = 0, 1, 2
 
 EXPORTS = ("csa2_page_bytes", "csa2_swa_bytes", "csa2_workspace_bytes", "csa2_prefill", "csa2_append",
            "csa2_index", "csa2_attend", "csa2_get_device_error", "csa2_status_string", "csa2_set_profile_events",
-           "csa2_launch_count")
+           "csa2_launch_count", "csa2_attend_noalloc")
+ATTEND_NOALLOC_MAX_ROWS = 512
 KERNEL_BLOCK_SCORE, KERNEL_FLAT_SCORE, KERNEL_POOL_SCORE, KERNEL_SELECT, KERNEL_ATTEND, KERNEL_COMBINE = range(6)
 
 
@@ -63,6 +64,7 @@ def _load():
         "csa2_get_device_error": (C.c_int, [P, C.POINTER(C.c_int32), P]),
         "csa2_status_string": (C.c_char_p, [C.c_int]),
         "csa2_set_profile_events": (C.c_int, [I32, P, P]),
+        "csa2_attend_noalloc": (C.c_int, [P, I32, P, P, C.c_float, P, I32, P]),
         "csa2_launch_count": (C.c_uint64, []),
     }
     for name, (res, args) in sig.items():
@@ -195,3 +197,18 @@ def csa2_set_profile_events(kernel: int, start=None, stop=None):
 
 def csa2_launch_count() -> int:
     return int(lib.csa2_launch_count())
+
+
+def csa2_attend_noalloc(cache: Cache, q, topk, scale: float, out, stream=None) -> int:
+    """csa2_attend without a workspace, for callers that cannot allocate
+    device memory: the library keeps the split partials in its own fixed
+    array (batch * heads <= ATTEND_NOALLOC_MAX_ROWS).  Returns the C status;
+    raises on anything but OK or CSA2_ERR_UNSUPPORTED (size over the limit)."""
+    heads = int(q.shape[1])
+    qq = q.view(torch.int16) if q.dtype == torch.bfloat16 else q
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    st = lib.csa2_attend_noalloc(cache.ref, heads, _ptr(qq), _ptr(topk), float(scale), _ptr(out), fp32,
+                                 _stream(stream))
+    if st not in (0, 2):
+        raise CSA2Error("csa2_attend_noalloc", st)
+    return int(st)

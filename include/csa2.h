@@ -192,6 +192,31 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
                         const int32_t *topk, float scale, void *out, int32_t out_is_fp32,
                         void *ws, size_t ws_bytes, csa2_stream_t stream);
 
+/* Attention without a workspace ------------------------------------------
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory -- for instance code embedded in a host
+ * framework that owns all device memory through its own pool and gives
+ * plugins no way to allocate, or a serving loop that must not allocate once
+ * it runs, because an allocation can synchronise the device.  It computes
+ * exactly what csa2_attend computes, with the same arguments minus ws and
+ * ws_bytes: the per-split partials live in one fixed array inside the
+ * library instead of a caller workspace.
+ *   - Limit: batch * heads <= CSA2_ATTEND_NOALLOC_MAX_ROWS (512).  Larger
+ *     calls return CSA2_ERR_UNSUPPORTED and enqueue nothing.
+ *   - The array (512 x 10 x 514 floats, about 10.5 MB) exists on every GPU
+ *     that loads the library and stays allocated until the process exits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.  No call allocates or frees memory.
+ *   - All calls share the one array and each overwrites every partial it
+ *     reads, so nothing carries over between calls; but two calls whose GPU
+ *     work can overlap (different streams, or concurrent host threads
+ *     without ordering) race on it -- order them on one stream. */
+#define CSA2_ATTEND_NOALLOC_MAX_ROWS 512
+csa2_status csa2_attend_noalloc(const csa2_cache *cache, int32_t heads, const uint16_t *q,
+                                const int32_t *topk, float scale, void *out, int32_t out_is_fp32,
+                                csa2_stream_t stream);
+
 /* Diagnostics ------------------------------------------------------------
  * Kernels that csa2_set_profile_events can bracket with CUDA events. */
 typedef enum {
