@@ -60,7 +60,8 @@ extern "C" csa2_status csa2_attend_noalloc(const csa2_cache *cache, int32_t head
         return CSA2_ERR_INVALID_ARG;
     if (cache->batch <= 0 || cache->n_pages <= 0 || cache->max_pages <= 0) return CSA2_ERR_INVALID_ARG;
     if (!aligned_to(cache->pool, 256) || !aligned_to(cache->swa, 256)) return CSA2_ERR_INVALID_ARG;
-    if (heads <= 0 || heads > 128 || !q || !topk || !out || !aligned_to(out, 16)) return CSA2_ERR_INVALID_ARG;
+    if (heads <= 0 || heads > 128 || !q || !topk || !out || !aligned_to(out, 16) || !aligned_to(q, 16))
+        return CSA2_ERR_INVALID_ARG;
     // The fixed array holds the partials of at most this many (request, head) rows.
     if ((int64_t)cache->batch * heads > CSA2_ATTEND_NOALLOC_MAX_ROWS) return CSA2_ERR_UNSUPPORTED;
     float *scratch = nullptr;

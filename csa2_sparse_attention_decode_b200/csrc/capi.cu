@@ -122,7 +122,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
 {
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
-    if (!q_idx || !w || !topk || !ws || !aligned(ws, 256)) return CSA2_ERR_INVALID_ARG;
+    if (!q_idx || !w || !topk || !ws || !aligned(ws, 256) || !aligned(q_idx, 16)) return CSA2_ERR_INVALID_ARG;
     if (mode != CSA2_INDEX_FLAT && mode != CSA2_INDEX_FULL && mode != CSA2_INDEX_REINDEX) return CSA2_ERR_INVALID_ARG;
     if (mode != CSA2_INDEX_FLAT && (!pool || !pool_len)) return CSA2_ERR_INVALID_ARG;
     const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
@@ -159,7 +159,7 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
     if (heads <= 0 || heads > 128 || !q || !topk || !out || !ws || !aligned(ws, 256)) return CSA2_ERR_INVALID_ARG;
-    if (!aligned(out, 16)) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16)) return CSA2_ERR_INVALID_ARG;
     const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
     Workspace W = layout(ws, cache->batch, heads, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;

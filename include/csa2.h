@@ -97,6 +97,7 @@ typedef enum {
 #define CSA2_DEV_CAPACITY        2   /* entry index >= max_pages * 64           */
 #define CSA2_DEV_BAD_INDEX       3   /* top-k / pool index outside the request  */
 #define CSA2_DEV_BAD_REQUEST     4   /* m not in {1,2}, n_new not in [0,2], ... */
+#define CSA2_DEV_TIMEOUT         5   /* a bounded in-kernel wait gave up        */
 
 typedef enum {
     CSA2_INDEX_FLAT = 0,     /* exact top-512 over every entry                   */
