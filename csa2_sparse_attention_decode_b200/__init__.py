@@ -20,7 +20,12 @@ LIB_PATH = os.path.join(_HERE, "libcsa2.so")
 LATENT, CODE_BYTES, SCALE_BYTES, KEY_DIM, IDX_HEADS = 512, 256, 32, 128, 32
 BLOCK, MAX_BLOCKS, POOL, TOPK, SWA = 8, 2048, 16384, 512, 128
 PAGE_ENTRIES, PAGE_BYTES, SWA_BYTES, PENDING_STRIDE = 64, 27648, 66048, 656
-PAGE_CODES_OFF, PAGE_SCALES_OFF, PAGE_KEYS_OFF, PAGE_SUMM_OFF = 0, 16384, 18432, 26624
+PAGE_CODES_BYTES, PAGE_SCALES_BYTES, PAGE_KEYS_BYTES, PAGE_SUMM_BYTES = 16384, 2048, 8192, 1024
+
+
+def plane_offsets(n_pages: int):
+    """Byte offsets of the codes / scales / keys / summaries planes of a pool."""
+    return 0, n_pages * 16384, n_pages * 18432, n_pages * 26624
 SWA_CODES_OFF, SWA_SCALE_OFF = 0, 65536
 INDEX_FLAT, INDEX_FULL, INDEX_REINDEX = 0, 1, 2
 

@@ -29,7 +29,7 @@ __device__ __forceinline__ void gate_weights(float g0, float g1, float &p0, floa
 __device__ __forceinline__ void pack_entry_warp(const float *lat0, const float *lat1,
                                                 const float *key0, const float *key1,
                                                 int m, float p0, float p1,
-                                                uint8_t *page, int slot, int lane)
+                                                const CacheView &c, int pid, int slot, int lane)
 {
     float x[16];
 #pragma unroll
@@ -56,9 +56,8 @@ __device__ __forceinline__ void pack_entry_warp(const float *lat0, const float *
 #pragma unroll
         for (int i = 0; i < 8; ++i) hi |= f32_to_e2m1(__fdiv_rn(x[8 + i], s)) << (4 * i);
     }
-    *reinterpret_cast<uint2 *>(page + CSA2_PAGE_CODES_OFF + slot * CSA2_CODE_BYTES + 8 * lane) =
-        make_uint2(lo, hi);
-    page[CSA2_PAGE_SCALES_OFF + slot * CSA2_SCALE_BYTES + lane] = sc;
+    *reinterpret_cast<uint2 *>(codes_row(c, pid, slot) + 8 * lane) = make_uint2(lo, hi);
+    scales_row(c, pid, slot)[lane] = sc;
 
     float4 k = *reinterpret_cast<const float4 *>(key0 + 4 * lane);
     if (m == 2) {
@@ -70,7 +69,7 @@ __device__ __forceinline__ void pack_entry_warp(const float *lat0, const float *
     }
     uint32_t kw = (uint32_t)f32_to_e4m3(k.x) | ((uint32_t)f32_to_e4m3(k.y) << 8) |
                   ((uint32_t)f32_to_e4m3(k.z) << 16) | ((uint32_t)f32_to_e4m3(k.w) << 24);
-    *reinterpret_cast<uint32_t *>(page + CSA2_PAGE_KEYS_OFF + slot * CSA2_KEY_DIM + 4 * lane) = kw;
+    *reinterpret_cast<uint32_t *>(keys_row(c, pid, slot) + 4 * lane) = kw;
 }
 
 // One warp quantises one raw token into its SWA slot.
@@ -107,13 +106,12 @@ __device__ __forceinline__ void block_summary(const CacheView &c, int b, int blk
 {
     int cnt = min(CSA2_BLOCK, n_entries - blk * CSA2_BLOCK);
     if (cnt <= 0) return;
-    uint8_t *page = entry_page(c, b, blk * CSA2_BLOCK);
-    if (!page) return;
+    const int pid = entry_pid(c, b, blk * CSA2_BLOCK);
+    if (pid < 0) return;
     int slot0 = (blk * CSA2_BLOCK) & (CSA2_PAGE_ENTRIES - 1);
     float sum = 0.0f;   // exact: e4m3 values are multiples of 2^-9 below 2^9
-    for (int j = 0; j < cnt; ++j)
-        sum += e4m3_to_f32(page[CSA2_PAGE_KEYS_OFF + (slot0 + j) * CSA2_KEY_DIM + i]);
-    page[CSA2_PAGE_SUMM_OFF + (blk & 7) * CSA2_KEY_DIM + i] = f32_to_e4m3(__fdiv_rn(sum, (float)cnt));
+    for (int j = 0; j < cnt; ++j) sum += e4m3_to_f32(keys_row(c, pid, slot0 + j)[i]);
+    summ_row(c, pid, blk & 7)[i] = f32_to_e4m3(__fdiv_rn(sum, (float)cnt));
 }
 
 // ------------------------------------------------------------------ prefill
@@ -126,14 +124,14 @@ __global__ void __launch_bounds__(256) prefill_entries_kernel(CacheView c, int r
     int le = blockIdx.x * 8 + w;
     if (le >= n_ent) return;
     int e = e_first + le;
-    uint8_t *page = entry_page(c, req, e);
-    if (!page) return;
+    const int pid = entry_pid(c, req, e);
+    if (pid < 0) return;
     int r0 = le * m;
     float p0 = 1.0f, p1 = 0.0f;
     if (m == 2) gate_weights(gate[r0], gate[r0 + 1], p0, p1);
     const float *l0 = lat + (size_t)r0 * CSA2_LATENT, *k0 = key + (size_t)r0 * CSA2_KEY_DIM;
-    pack_entry_warp(l0, l0 + CSA2_LATENT, k0, k0 + CSA2_KEY_DIM, m, p0, p1, page,
-                    e & (CSA2_PAGE_ENTRIES - 1), lane);
+    pack_entry_warp(l0, l0 + CSA2_LATENT, k0, k0 + CSA2_KEY_DIM, m, p0, p1, c, pid, e & (CSA2_PAGE_ENTRIES - 1),
+                    lane);
 }
 
 __global__ void __launch_bounds__(128) prefill_summary_kernel(CacheView c, int req, int blk_first, int n_entries)
@@ -175,6 +173,8 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const float *l
     __shared__ int s_ent[2];
     int b = blockIdx.x;
     int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dependency_wait();
+    allow_dependents();
     int n0 = c.n_tokens[b];
     int m = c.m[b];
     int k = n_new_arr[b];
@@ -210,13 +210,13 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const float *l
     if (w >= 2 && w - 2 < n_ent) {
         int i = w - 2;
         int e = e0 + i;
-        uint8_t *page = entry_page(c, b, e);
-        if (page) {
+        const int pid = entry_pid(c, b, e);
+        if (pid >= 0) {
             const float *t0 = &s_tok[i * m][0];
             const float *t1 = (m == 2) ? &s_tok[i * m + 1][0] : t0;
             float p0 = 1.0f, p1 = 0.0f;
             if (m == 2) gate_weights(t0[CSA2_LATENT + CSA2_KEY_DIM], t1[CSA2_LATENT + CSA2_KEY_DIM], p0, p1);
-            pack_entry_warp(t0, t1, t0 + CSA2_LATENT, t1 + CSA2_LATENT, m, p0, p1, page,
+            pack_entry_warp(t0, t1, t0 + CSA2_LATENT, t1 + CSA2_LATENT, m, p0, p1, c, pid,
                             e & (CSA2_PAGE_ENTRIES - 1), lane);
         }
     }
@@ -269,8 +269,7 @@ cudaError_t launch_append(const CacheView &c, const float *lat, const float *key
                           const int32_t *n_new, cudaStream_t st)
 {
     LaunchScope scope(-1, st);
-    append_kernel<<<c.batch, 256, 0, st>>>(c, lat, key, gate, n_new);
-    return cudaGetLastError();
+    return launch_pdl(append_kernel, dim3(c.batch), dim3(256), 0, st, c, lat, key, gate, n_new);
 }
 
 }  // namespace csa2

@@ -7,8 +7,9 @@
 // channels; fp8 SWA with a 128-token window).
 //
 // One CTA per (request, 128-key tile, 64-head group); tiles 0-3 are the
-// top-512 entries, tile 4 the SWA window.  128 threads; thread i owns key row
-// i while loading and row i of every tensor-memory tile afterwards.
+// top-512 entries, tile 4 the SWA window.  256 threads; threads i and i+128
+// share key row i (each half of its channels / heads) while loading and
+// tensor-memory row i afterwards.
 //   1. q (bf16, 64 heads x 512) -> smem, K-major, 128-byte swizzle.
 //   2. gather + dequantise 128 keys to bf16 (exact: e2m1 x e4m3 and
 //      e4m3 x 2^e all fit bf16) -> smem V tile, K-major, swizzled.
@@ -18,13 +19,19 @@
 //      the second product keeps ~16 bits of P.
 //   5. O^T[512 x 64] = V^T . (P_hi + P_lo)^T       (4 x 16 MMAs; V reused as
 //      an MN-major operand, P as MN-major [key][head])
-//   6. partials: m[h], l[h] = sum_j p_j, o[h][d] = sum_j p_j v_j (fp32).
-// A log-sum-exp combine merges the 5 tiles per request.
+//   6. the five tiles of a (request, head group) form one thread-block
+//      cluster: they exchange the per-head max m and sum l over distributed
+//      shared memory, write their partial o scaled by exp(m_tile - M) / L to
+//      the workspace, and each CTA then sums one fifth of the output.
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "index.cuh"
 #include "umma.cuh"
+
+#include <cooperative_groups.h>
+namespace cg = cooperative_groups;
 
 namespace csa2 {
 using namespace umma;
@@ -33,7 +40,8 @@ namespace {
 
 constexpr int KT = 128;                    // keys per tile
 constexpr int HG = 64;                     // heads per CTA
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;
+constexpr int NTILES = ATT_SPLITS;         // 4 top-k tiles + the window = one cluster
 constexpr int V_SLAB = KT * 128;           // 16 KB: 128 rows x 64 bf16
 constexpr int V_BYTES = 8 * V_SLAB;        // 128 KB
 constexpr int Q_SLAB = HG * 128;           // 8 KB
@@ -95,124 +103,128 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
     return false;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-attend_umma_kernel(CacheView c, int heads, const uint16_t *q, const int32_t *topk, float scale, float *part_o,
-                   float *part_ml)
+__global__ void __cluster_dims__(NTILES, 1, 1) __launch_bounds__(THREADS, 1)
+attend_umma_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads, const int32_t *topk, float scale,
+                   void *out, int out_is_fp32, float *part_o)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *Vs = sm, *Qs = sm + V_BYTES;
     float *Ts = reinterpret_cast<float *>(Qs + T_OFF);
-    __shared__ __align__(8) uint64_t bar_s, bar_o;
+    __shared__ __align__(8) uint64_t bar_q, bar_s, bar_o;
     __shared__ uint32_t tmem_base;
-    __shared__ float m_s[HG], l_s[HG], red_s[2][HG];
-    __shared__ int any_valid;
+    __shared__ float m_s[HG], l_s[HG], fac_s[HG], red_s[4][HG];
+    __shared__ int any_valid, tile_live[NTILES];
+    cg::cluster_group cluster = cg::this_cluster();
 
     const int tile = blockIdx.x, hg0 = blockIdx.y * HG, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & (KT - 1), half = tid >> 7;      // two threads per key / tensor-memory row
+    if (warp == 0) tmem_alloc(&tmem_base, TMEM_COLS);
+    if (tid == 32) tma_prefetch_map(&map_q);
+    grid_dependency_wait();                               // q, top-k and the cache may be fresh
+    allow_dependents();
     const int n_tok = c.n_tokens[b];
     const int n_entries = n_entries_of(c, b);
     const int nv = max(0, min(n_tok, CSA2_SWA));
     const int nh = min(HG, heads - hg0);
 
-    if (warp == 0) tmem_alloc(&tmem_base, TMEM_COLS);
     if (tid == 0) {
+        mbar_init(&bar_q, 1);
         mbar_init(&bar_s, 1);
         mbar_init(&bar_o, 1);
-        any_valid = 0;
         mbar_fence_init();
+        // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x 64 heads, 128-byte
+        // swizzled (K-major operand layout); heads past `heads` read as zero.
+        mbar_arrive_expect_tx(&bar_q, Q_BYTES);
+        for (int slab = 0; slab < 8; ++slab) tma_load_3d(Qs + slab * Q_SLAB, &map_q, 64 * slab, hg0, b, &bar_q);
     }
+    if (tid == 1) any_valid = 0;
+    __syncthreads();
 
-    // ---- 1. q -> smem (K-major, swizzled); rows past `heads` are zero
-    for (int i = tid; i < HG * 64; i += THREADS) {
-        const int h = i >> 6, cidx = i & 63;               // cidx = 16-byte chunk along the 512 dims
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (h < nh) v = *reinterpret_cast<const uint4 *>(q + ((size_t)b * heads + hg0 + h) * CSA2_LATENT + 8 * cidx);
-        const int slab = cidx >> 3, ch = cidx & 7;
-        *reinterpret_cast<uint4 *>(Qs + slab * Q_SLAB + h * 128 + ((ch ^ (h & 7)) << 4)) = v;
-    }
-
-    // ---- 2. key row tid -> bf16, K-major swizzled (8 slabs of 64 channels)
+    // ---- 2. key `row`, channels [256*half, 256*half + 256) -> bf16 in slabs 4*half .. 4*half+3
     bool valid = false;
-    const int r = tid;
     if (tile < CSA2_TOPK / KT) {
-        const int e = topk[(size_t)b * CSA2_TOPK + tile * KT + r];
-        if (e >= n_entries) set_error(c.error, CSA2_DEV_BAD_INDEX);
-        const uint8_t *pg = (e >= 0 && e < n_entries) ? entry_page(c, b, e) : nullptr;
-        if (pg) {
+        const int e = topk[(size_t)b * CSA2_TOPK + tile * KT + row];
+        if (e >= n_entries && half == 0) set_error(c.error, CSA2_DEV_BAD_INDEX);
+        const int pid = (e >= 0 && e < n_entries) ? entry_pid(c, b, e) : -1;
+        if (pid >= 0) {
             valid = true;
             const int slot = e & (CSA2_PAGE_ENTRIES - 1);
-            const uint4 *codes = reinterpret_cast<const uint4 *>(pg + CSA2_PAGE_CODES_OFF + slot * CSA2_CODE_BYTES);
-            const uint4 *scl = reinterpret_cast<const uint4 *>(pg + CSA2_PAGE_SCALES_OFF + slot * CSA2_SCALE_BYTES);
-            uint4 sv[2] = {scl[0], scl[1]};
-            const uint8_t *sb = reinterpret_cast<const uint8_t *>(sv);
-#pragma unroll 2
-            for (int slab = 0; slab < 8; ++slab) {
-                uint4 cw[2] = {codes[2 * slab], codes[2 * slab + 1]};          // 64 channels
-                const uint32_t *cwu = reinterpret_cast<const uint32_t *>(cw);
+            const uint4 *codes = reinterpret_cast<const uint4 *>(codes_row(c, pid, slot)) + 8 * half;
+            const uint4 sv = reinterpret_cast<const uint4 *>(scales_row(c, pid, slot))[half];
+            uint4 cw[8];                               // 128 code bytes, loads issued together
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cw[i] = codes[i];
+            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                const int slab = 4 * half + s4;
+                const uint32_t cwu[8] = {cw[2 * s4].x,     cw[2 * s4].y,     cw[2 * s4].z,     cw[2 * s4].w,
+                                         cw[2 * s4 + 1].x, cw[2 * s4 + 1].y, cw[2 * s4 + 1].z, cw[2 * s4 + 1].w};
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {                                  // 8 channels per chunk
                     uint32_t o[4];
                     e2m1x8_to_bf16(cwu[ch], o);
-                    // channels slab*64 + ch*8 .. +7 share scale (slab*64 + ch*8) / 16
-                    const float sf = e4m3_to_f32(sb[slab * 4 + (ch >> 1)]);
-                    const __nv_bfloat16 s16 = __float2bfloat16_rn(sf);
-                    const uint32_t s2 = (uint32_t)__bfloat16_as_ushort(s16) * 0x10001u;
+                    // channels slab*64 + ch*8 .. +7 share scale byte slab*4 + ch/2
+                    const int si = s4 * 4 + (ch >> 1);
+                    const float sf = e4m3_to_f32((uint8_t)(sw[si >> 2] >> (8 * (si & 3))));
+                    const uint32_t s2 = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(sf)) * 0x10001u;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) o[i] = bf16x2_mul(o[i], s2);
-                    *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                    *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + ((ch ^ (row & 7)) << 4)) =
                         make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
         }
-    } else if (r < nv) {
+    } else if (row < nv) {
         valid = true;
-        const uint8_t *sw = swa_base(c, b);
-        const float sc = reinterpret_cast<const float *>(sw + CSA2_SWA_SCALE_OFF)[r];
-        const uint4 *codes = reinterpret_cast<const uint4 *>(sw + CSA2_SWA_CODES_OFF + r * CSA2_LATENT);
-#pragma unroll 2
-        for (int slab = 0; slab < 8; ++slab) {
+        const uint8_t *swa = swa_base(c, b);
+        const float sc = reinterpret_cast<const float *>(swa + CSA2_SWA_SCALE_OFF)[row];
+        const uint4 *codes = reinterpret_cast<const uint4 *>(swa + CSA2_SWA_CODES_OFF + row * CSA2_LATENT) + 16 * half;
+        uint4 cv[16];
 #pragma unroll
-            for (int half = 0; half < 4; ++half) {                              // 16 codes -> 2 chunks
-                uint4 cv = codes[slab * 4 + half];
-                const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-                uint32_t o[8];
+        for (int i = 0; i < 16; ++i) cv[i] = codes[i];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] & 0xffff), __NV_E4M3);
-                    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] >> 16), __NV_E4M3);
-                    __nv_bfloat162 a = __floats2bfloat162_rn(__half2float(__ushort_as_half(lo.x)) * sc,
-                                                             __half2float(__ushort_as_half(lo.y)) * sc);
-                    __nv_bfloat162 bq = __floats2bfloat162_rn(__half2float(__ushort_as_half(hi.x)) * sc,
-                                                              __half2float(__ushort_as_half(hi.y)) * sc);
-                    o[2 * i] = *reinterpret_cast<uint32_t *>(&a);
-                    o[2 * i + 1] = *reinterpret_cast<uint32_t *>(&bq);
-                }
-                const int ch0 = 2 * half;
-                *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + r * 128 + ((ch0 ^ (r & 7)) << 4)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + r * 128 + (((ch0 + 1) ^ (r & 7)) << 4)) =
-                    make_uint4(o[4], o[5], o[6], o[7]);
+        for (int k = 0; k < 16; ++k) {                                          // 16 codes -> 2 chunks
+            const int slab = 4 * half + (k >> 2), ch0 = 2 * (k & 3);
+            const uint32_t cw[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] & 0xffff), __NV_E4M3);
+                __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] >> 16), __NV_E4M3);
+                __nv_bfloat162 a = __floats2bfloat162_rn(__half2float(__ushort_as_half(lo.x)) * sc,
+                                                         __half2float(__ushort_as_half(lo.y)) * sc);
+                __nv_bfloat162 bq = __floats2bfloat162_rn(__half2float(__ushort_as_half(hi.x)) * sc,
+                                                          __half2float(__ushort_as_half(hi.y)) * sc);
+                o[2 * i] = *reinterpret_cast<uint32_t *>(&a);
+                o[2 * i + 1] = *reinterpret_cast<uint32_t *>(&bq);
             }
+            *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + ((ch0 ^ (row & 7)) << 4)) =
+                make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + (((ch0 + 1) ^ (row & 7)) << 4)) =
+                make_uint4(o[4], o[5], o[6], o[7]);
         }
     }
     if (!valid) {
-        for (int slab = 0; slab < 8; ++slab)
+        for (int s4 = 0; s4 < 4; ++s4)
             for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + r * 128 + (ch << 4)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(Vs + (4 * half + s4) * V_SLAB + row * 128 + (ch << 4)) =
+                    make_uint4(0, 0, 0, 0);
     }
     if (valid) any_valid = 1;
     fence_proxy_async_smem();
     __syncthreads();
     fence_after_sync();
     const uint32_t tb = tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const bool live = any_valid != 0;
-    float *pml = part_ml + ((size_t)b * ATT_SPLITS + tile) * heads * 2;
 
     if (live) {
         // ---- 3. S^T = V . Q^T
         if (tid == 0) {
+            wait_bar(&bar_q, 0, c.error);
             const uint32_t va = smem_addr(Vs), qa = smem_addr(Qs);
 #pragma unroll 4
             for (int kk = 0; kk < CSA2_LATENT / 16; ++kk) {
@@ -226,50 +238,47 @@ attend_umma_kernel(CacheView c, int heads, const uint16_t *q, const int32_t *top
         wait_bar(&bar_s, 0, c.error);
         fence_after_sync();
 
-        // ---- 4. softmax over this tile's keys, per head
-        float lg[HG];
+        // ---- 4. softmax over the tile's keys, per head (thread: key `row`, heads 32*half ..)
+        float lg[32];
         {
             uint32_t rr[32];
+            tmem_ld32(tb + lane_base + S_COL + 32 * half, rr);
+            tmem_ld_wait();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tb + lane_base + S_COL + 32 * half, rr);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) lg[32 * half + j] = valid ? __uint_as_float(rr[j]) * scale : -INFINITY;
-            }
+            for (int j = 0; j < 32; ++j) lg[j] = valid ? __uint_as_float(rr[j]) * scale : -INFINITY;
         }
-        // q smem is free from here on (the product above has completed).
+        // the q region is free from here on (the product above has completed)
 #pragma unroll
-        for (int h = 0; h < HG; ++h) Ts[r * T_STRIDE + h] = lg[h];
+        for (int j = 0; j < 32; ++j) Ts[row * T_STRIDE + 32 * half + j] = lg[j];
         __syncthreads();
         {
             const int h = tid & (HG - 1), part = tid >> 6;
             float mx = -INFINITY;
-            for (int j = part * 64; j < part * 64 + 64; ++j) mx = fmaxf(mx, Ts[j * T_STRIDE + h]);
+            for (int j = part * 32; j < part * 32 + 32; ++j) mx = fmaxf(mx, Ts[j * T_STRIDE + h]);
             red_s[part][h] = mx;
         }
         __syncthreads();
-        if (tid < HG) m_s[tid] = fmaxf(red_s[0][tid], red_s[1][tid]);
+        if (tid < HG) m_s[tid] = fmaxf(fmaxf(red_s[0][tid], red_s[1][tid]), fmaxf(red_s[2][tid], red_s[3][tid]));
         __syncthreads();
         uint8_t *Ph = Qs + PHI_OFF, *Pl = Qs + PLO_OFF;
 #pragma unroll
-        for (int cch = 0; cch < 8; ++cch) {
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const int cch = 4 * half + c4;                 // 8-head chunk of the P row
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int h0 = 8 * cch + 2 * i;
-                const float m0 = m_s[h0], m1 = m_s[h0 + 1];
-                const float p0 = valid ? __expf(lg[h0] - m0) : 0.0f;
-                const float p1 = valid ? __expf(lg[h0 + 1] - m1) : 0.0f;
-                Ts[r * T_STRIDE + h0] = p0;
-                Ts[r * T_STRIDE + h0 + 1] = p1;
+                const int j0 = 8 * c4 + 2 * i, h0 = 32 * half + j0;
+                const float p0 = valid ? __expf(lg[j0] - m_s[h0]) : 0.0f;
+                const float p1 = valid ? __expf(lg[j0 + 1] - m_s[h0 + 1]) : 0.0f;
+                Ts[row * T_STRIDE + h0] = p0;
+                Ts[row * T_STRIDE + h0 + 1] = p1;
                 const __nv_bfloat162 ph = __floats2bfloat162_rn(p0, p1);
                 const float2 phf = __bfloat1622float2(ph);
                 const __nv_bfloat162 pl = __floats2bfloat162_rn(p0 - phf.x, p1 - phf.y);
                 hi[i] = *reinterpret_cast<const uint32_t *>(&ph);
                 lo[i] = *reinterpret_cast<const uint32_t *>(&pl);
             }
-            const uint32_t off = r * 128 + ((cch ^ (r & 7)) << 4);
+            const uint32_t off = row * 128 + ((cch ^ (row & 7)) << 4);
             *reinterpret_cast<uint4 *>(Ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4 *>(Pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
@@ -297,37 +306,79 @@ attend_umma_kernel(CacheView c, int heads, const uint16_t *q, const int32_t *top
         {
             const int h = tid & (HG - 1), part = tid >> 6;
             float sum = 0.0f;
-            for (int j = part * 64; j < part * 64 + 64; ++j) sum += Ts[j * T_STRIDE + h];
+            for (int j = part * 32; j < part * 32 + 32; ++j) sum += Ts[j * T_STRIDE + h];
             red_s[part][h] = sum;
         }
         __syncthreads();
-        if (tid < nh) {
-            l_s[tid] = red_s[0][tid] + red_s[1][tid];
-            pml[(size_t)(hg0 + tid) * 2] = m_s[tid];
-            pml[(size_t)(hg0 + tid) * 2 + 1] = l_s[tid];
+        if (tid < HG) l_s[tid] = (red_s[0][tid] + red_s[1][tid]) + (red_s[2][tid] + red_s[3][tid]);
+    } else {
+        if (tid == 0) wait_bar(&bar_q, 0, c.error);          // no copy may be in flight at exit
+        if (tid < HG) {
+            m_s[tid] = -INFINITY;
+            l_s[tid] = 0.0f;
         }
+    }
+    // ---- 6. combine the five tiles of this (request, head group) in-cluster:
+    // exchange (m, l) over distributed shared memory; each tile writes its
+    // partial already scaled by exp(m_tile - M) / L; then each CTA sums one
+    // fifth of the output over the live tiles.
+    cluster.sync();
+    if (tid < HG) {
+        float mr[NTILES], M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < NTILES; ++r) {
+            mr[r] = cluster.map_shared_rank(&m_s[0], r)[tid];
+            M = fmaxf(M, mr[r]);
+        }
+        float L = 0.0f;
+#pragma unroll
+        for (int r = 0; r < NTILES; ++r)
+            if (mr[r] != -INFINITY) L += __expf(mr[r] - M) * cluster.map_shared_rank(&l_s[0], r)[tid];
+        fac_s[tid] = (live && M != -INFINITY && L > 0.0f) ? __expf(m_s[tid] - M) / L : 0.0f;
+        if (tid < NTILES) tile_live[tid] = cluster.map_shared_rank(&m_s[0], tid)[0] != -INFINITY;
+    }
+    __syncthreads();
+    if (live) {
         wait_bar(&bar_o, 0, c.error);
         fence_after_sync();
-        // ---- 6. partial outputs: thread = latent row within each 128-chunk
         for (int cc = 0; cc < 4; ++cc) {
             uint32_t rr[32];
+            tmem_ld32(tb + lane_base + O_COL + 64 * cc + 32 * half, rr);
+            tmem_ld_wait();
+            const int d = 128 * cc + row;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tb + lane_base + O_COL + 64 * cc + 32 * half, rr);
-                tmem_ld_wait();
-                const int d = 128 * cc + tid;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int h = 32 * half + j;
-                    if (h < nh)
-                        part_o[(((size_t)b * ATT_SPLITS + tile) * heads + hg0 + h) * CSA2_LATENT + d] =
-                            __uint_as_float(rr[j]);
-                }
+            for (int j = 0; j < 32; ++j) {
+                const int h = 32 * half + j;
+                if (h < nh)
+                    part_o[(((size_t)b * NTILES + tile) * heads + hg0 + h) * CSA2_LATENT + d] =
+                        __uint_as_float(rr[j]) * fac_s[h];
             }
         }
-    } else if (tid < nh) {
-        pml[(size_t)(hg0 + tid) * 2] = -INFINITY;
-        pml[(size_t)(hg0 + tid) * 2 + 1] = 0.0f;
+    }
+    cluster.sync();                                       // partials visible cluster-wide
+    {
+        const int total4 = HG * (CSA2_LATENT / 4);
+        const int lo4 = tile * total4 / NTILES, hi4 = (tile + 1) * total4 / NTILES;
+        for (int i = lo4 + tid; i < hi4; i += THREADS) {
+            const int h = i / (CSA2_LATENT / 4), d4 = i % (CSA2_LATENT / 4);
+            if (h >= nh) continue;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < NTILES; ++r) {
+                if (!tile_live[r]) continue;
+                const float4 v = *reinterpret_cast<const float4 *>(
+                    part_o + (((size_t)b * NTILES + r) * heads + hg0 + h) * CSA2_LATENT + 4 * d4);
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            const size_t o = ((size_t)b * heads + hg0 + h) * CSA2_LATENT + 4 * d4;
+            if (out_is_fp32) {
+                *reinterpret_cast<float4 *>((float *)out + o) = acc;
+            } else {
+                __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+                uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+                *reinterpret_cast<uint2 *>((__nv_bfloat16 *)out + o) = pk;
+            }
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -337,10 +388,25 @@ attend_umma_kernel(CacheView c, int heads, const uint16_t *q, const int32_t *top
     }
 }
 
+// q viewed as a 3-D bf16 tensor (512 dims, heads, batch); boxes of 64 dims x
+// 64 heads, 128-byte swizzled.
+bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch)
+{
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {CSA2_LATENT, (cuuint64_t)heads, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {CSA2_LATENT * 2, (cuuint64_t)heads * CSA2_LATENT * 2};
+    cuuint32_t box[3] = {64, HG, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)q, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                               float *part_o, float *part_ml, cudaStream_t st)
+                               void *out, int out_is_fp32, float *part_o, cudaStream_t st)
 {
     static bool attr_done[64] = {};
     int dev = 0;
@@ -351,10 +417,12 @@ cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q,
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done[dev] = true;
     }
-    dim3 grid(ATT_SPLITS, (heads + HG - 1) / HG, c.batch);
+    CUtensorMap map_q;
+    if (!make_q_map(&map_q, q, heads, c.batch)) return cudaErrorInvalidValue;
+    dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);
     LaunchScope scope(CSA2_KERNEL_ATTEND, st);
-    attend_umma_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(c, heads, q, topk, scale, part_o, part_ml);
-    return cudaGetLastError();
+    return launch_pdl(attend_umma_kernel, grid, dim3(THREADS), SMEM_BYTES, st, map_q, c, heads, topk, scale, out,
+                      out_is_fp32, part_o);
 }
 
 }  // namespace csa2

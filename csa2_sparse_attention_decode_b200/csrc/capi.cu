@@ -135,7 +135,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
         e = launch_score(c, ROWS_KEYS, q_idx, w, nullptr, nullptr, W.scores_a, W.row_stride, max_entries, s);
         if (e == cudaSuccess)
             e = launch_select(c, ROWS_KEYS, W.scores_a, W.row_stride, nullptr, nullptr, CSA2_TOPK, topk, CSA2_TOPK,
-                              0, nullptr, nullptr, s);
+                              0, nullptr, nullptr, max_entries, s);
         return from_cuda(e);
     }
     if (mode == CSA2_INDEX_FULL) {
@@ -143,13 +143,13 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
         e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores_a, W.row_stride, max_blocks, s);
         if (e == cudaSuccess)
             e = launch_select(c, ROWS_SUMMARIES, W.scores_a, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS,
-                              W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, s);
+                              W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, max_blocks, s);
         if (e != cudaSuccess) return from_cuda(e);
     }
     e = launch_score(c, ROWS_POOL, q_idx, w, pool, pool_len, W.scores_b, CSA2_POOL, CSA2_POOL, s);
     if (e == cudaSuccess)
         e = launch_select(c, ROWS_POOL, W.scores_b, CSA2_POOL, pool_len, pool, CSA2_TOPK, topk, CSA2_TOPK, 0,
-                          nullptr, nullptr, s);
+                          nullptr, nullptr, CSA2_POOL, s);
     return from_cuda(e);
 }
 

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/csa2.h"
 
 namespace csa2 {
@@ -21,6 +23,30 @@ struct LaunchScope {
     LaunchScope(int kernel, cudaStream_t s) : k(kernel), st(s) { note_launch(k, st, true); }
     ~LaunchScope() { note_launch(k, st, false); }
 };
+
+// ---------------------------------------------------------------- launch order
+// Programmatic dependent launch: every kernel lets the next one in the
+// stream start its launch and set-up early, and waits for the previous one
+// (completion and memory) before touching anything it may have written.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- errors
 __device__ __forceinline__ void set_error(int32_t *err, int32_t code)
@@ -70,6 +96,7 @@ __device__ __forceinline__ int swa_exponent(float amax)
 // ---------------------------------------------------------------- layout
 struct CacheView {
     uint8_t *pool;
+    uint8_t *codes, *scales, *keys, *summ;     // the four planes of the pool
     int32_t n_pages;
     const int32_t *page_table;
     int32_t max_pages;
@@ -85,6 +112,10 @@ __host__ inline CacheView make_view(const csa2_cache *c)
 {
     CacheView v;
     v.pool = (uint8_t *)c->pool;
+    v.codes = v.pool + CSA2_PLANE_CODES(c->n_pages);
+    v.scales = v.pool + CSA2_PLANE_SCALES(c->n_pages);
+    v.keys = v.pool + CSA2_PLANE_KEYS(c->n_pages);
+    v.summ = v.pool + CSA2_PLANE_SUMM(c->n_pages);
     v.n_pages = c->n_pages;
     v.page_table = c->page_table;
     v.max_pages = c->max_pages;
@@ -97,21 +128,39 @@ __host__ inline CacheView make_view(const csa2_cache *c)
     return v;
 }
 
-// Page base of entry e (or block e/8) of request b; nullptr (and the error
-// word set) when the page slot or page id is out of range.
-__device__ __forceinline__ uint8_t *entry_page(const CacheView &c, int b, int e)
+// Page id of entry e (or of block e/8) of request b; -1 (and the error word
+// set) when the page slot or the page id is out of range.
+__device__ __forceinline__ int entry_pid(const CacheView &c, int b, int e)
 {
     int pi = e >> 6;
     if (e < 0 || pi >= c.max_pages) {
         set_error(c.error, CSA2_DEV_CAPACITY);
-        return nullptr;
+        return -1;
     }
     int pid = __ldg(c.page_table + (size_t)b * c.max_pages + pi);
     if (pid < 0 || pid >= c.n_pages) {
         set_error(c.error, CSA2_DEV_BAD_PAGE);
-        return nullptr;
+        return -1;
     }
-    return c.pool + (size_t)pid * CSA2_PAGE_BYTES;
+    return pid;
+}
+
+// Field rows of entry slot `slot` (0..63) / summary slot (0..7) of page pid.
+__device__ __forceinline__ uint8_t *codes_row(const CacheView &c, int pid, int slot)
+{
+    return c.codes + (size_t)pid * CSA2_PAGE_CODES_BYTES + slot * CSA2_CODE_BYTES;
+}
+__device__ __forceinline__ uint8_t *scales_row(const CacheView &c, int pid, int slot)
+{
+    return c.scales + (size_t)pid * CSA2_PAGE_SCALES_BYTES + slot * CSA2_SCALE_BYTES;
+}
+__device__ __forceinline__ uint8_t *keys_row(const CacheView &c, int pid, int slot)
+{
+    return c.keys + (size_t)pid * CSA2_PAGE_KEYS_BYTES + slot * CSA2_KEY_DIM;
+}
+__device__ __forceinline__ uint8_t *summ_row(const CacheView &c, int pid, int sslot)
+{
+    return c.summ + (size_t)pid * CSA2_PAGE_SUMM_BYTES + sslot * CSA2_KEY_DIM;
 }
 
 __device__ __forceinline__ uint8_t *swa_base(const CacheView &c, int b)

@@ -46,7 +46,8 @@ __device__ __forceinline__ uint32_t scan256(uint32_t v, uint32_t *scratch)
     return v + add;
 }
 
-// One cluster of 8 CTAs per request (grid = 8 x batch).  Selects the top
+// One cluster of NC CTAs per request (grid = NC x batch; NC = 1 is a plain
+// CTA and uses no cluster barriers).  Selects the top
 // min(k, n) of scores[b][0..n) -- score descending, ties to the lower index --
 // and writes the selected ids in ascending order to out[b][0..k) (-1 padded).
 // The id of element i is i, or ids[b][i] when ids != nullptr.  With expand the
@@ -58,28 +59,38 @@ __device__ __forceinline__ uint32_t scan256(uint32_t v, uint32_t *scratch)
 // memory when chunk > SEL_CAP).  Four 8-bit radix passes find the exact
 // threshold key T and how many ties at T to keep; the per-CTA histograms and
 // the final per-CTA counts are exchanged through distributed shared memory.
-__global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREADS, 1)
-select_cluster_kernel(CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,
+template <int NC>
+__device__ __forceinline__ void select_body(CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,
                       const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
                       int32_t *pool_len)
 {
     extern __shared__ uint32_t keys[];
     __shared__ uint32_t hist[2][256];
+    __shared__ uint32_t whist[32][256];
     __shared__ uint32_t scratch[32];
     __shared__ uint32_t wsum[32][2];
     __shared__ uint32_t s_cnt[2];
     __shared__ uint32_t s_digit, s_above;
-    cg::cluster_group cluster = cg::this_cluster();
-    const int rank = (int)cluster.block_rank();
+    const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
+    auto csync = [&]() {
+        if constexpr (NC > 1) cg::this_cluster().sync();
+        else __syncthreads();
+    };
+    auto remote = [&](uint32_t *ptr, int r) -> uint32_t * {
+        if constexpr (NC > 1) return cg::this_cluster().map_shared_rank(ptr, r);
+        else return ptr;
+    };
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    grid_dependency_wait();                      // scores come from the previous kernel
+    allow_dependents();
     const int n_entries = n_entries_of(c, b);
     const int n = (src == ROWS_KEYS) ? n_entries
                 : (src == ROWS_SUMMARIES) ? (n_entries + CSA2_BLOCK - 1) / CSA2_BLOCK
                                           : max(0, min(pool_len_in[b], CSA2_POOL));
     const int kk = min(k, n);
     const bool take_all = n <= k;
-    const int chunk = (n + SEL_CLUSTER - 1) / SEL_CLUSTER;
+    const int chunk = (n + NC - 1) / NC;
     const int lo = rank * chunk;
     const int cnt = max(0, min(n, lo + chunk) - lo);
     const bool in_smem = chunk <= SEL_CAP;
@@ -87,13 +98,29 @@ select_cluster_kernel(CacheView c, int src, const float *scores, int64_t score_s
     const float *s = scores + (size_t)b * score_stride + lo;
     auto key_at = [&](int e) -> uint32_t { return in_smem ? keys[e] : ord_key(s[e]); };
 
-    if (in_smem)
-        for (int e = tid; e < cnt; e += SEL_THREADS) keys[e] = ord_key(s[e]);
+    if (in_smem) {
+        // 8 independent loads in flight per thread per round.
+        for (int e0 = 0; e0 < cnt; e0 += 8 * SEL_THREADS) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * SEL_THREADS + tid;
+                v[u] = e < cnt ? s[e] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * SEL_THREADS + tid;
+                if (e < cnt) keys[e] = ord_key(v[u]);
+            }
+        }
+    }
     uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kk;
     if (!take_all) {
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass, buf = pass & 1;
-            if (tid < 256) hist[buf][tid] = 0;
+            // Per-warp histograms: the leading digits of nearby scores are all
+            // equal, so one shared counter would serialise every warp.
+            for (int i = tid; i < 32 * 256; i += SEL_THREADS) whist[i >> 8][i & 255] = 0;
             __syncthreads();
             for (int it = 0; it < seg; it += 32) {
                 const int e = wid * seg + it + lane;
@@ -101,15 +128,35 @@ select_cluster_kernel(CacheView c, int src, const float *scores, int64_t score_s
                 const uint32_t key = valid ? key_at(e) : 0u;
                 const bool match = valid && (key & pmask) == prefix;
                 const uint32_t dig = (key >> shift) & 255u;
-                const uint32_t mm = __match_any_sync(0xffffffffu, match ? dig : 0x100u + lane);
-                if (match && (__ffs(mm) - 1) == lane) atomicAdd(&hist[buf][dig], (uint32_t)__popc(mm));
+                // Usually every matching lane has the same digit: one add by
+                // lane 0; otherwise shared-memory atomics on this warp's copy.
+                const uint32_t mb = __ballot_sync(0xffffffffu, match);
+                const uint32_t d0 = __shfl_sync(0xffffffffu, dig, mb ? __ffs(mb) - 1 : 0);
+                if (__all_sync(0xffffffffu, !match || dig == d0)) {
+                    if (lane == 0 && mb) whist[wid][d0] += (uint32_t)__popc(mb);
+                } else if (match) {
+                    atomicAdd(&whist[wid][dig], 1u);
+                }
+                __syncwarp();
             }
             __syncthreads();
-            cluster.sync();
+            if (tid < 256) {
+                uint32_t t = 0;
+#pragma unroll 8
+                for (int w = 0; w < 32; ++w) t += whist[w][tid];
+                hist[buf][tid] = t;
+            }
+            __syncthreads();
+            csync();
             // Cluster-wide count of bin 255 - tid, then counts of bins >= it.
             uint32_t hv = 0;
-            if (tid < 256)
-                for (int r = 0; r < SEL_CLUSTER; ++r) hv += cluster.map_shared_rank(&hist[buf][0], r)[255 - tid];
+            if (tid < 256) {
+                uint32_t part[NC];
+#pragma unroll
+                for (int r = 0; r < NC; ++r) part[r] = remote(&hist[buf][0], r)[255 - tid];
+#pragma unroll
+                for (int r = 0; r < NC; ++r) hv += part[r];
+            }
             const uint32_t incl = scan256(hv, scratch);
             if (tid < 256 && incl >= krem && incl - hv < krem) {
                 s_digit = 255u - tid;
@@ -149,10 +196,10 @@ select_cluster_kernel(CacheView c, int src, const float *scores, int64_t score_s
         s_cnt[1] = q;
     }
     __syncthreads();
-    cluster.sync();
+    csync();
     uint32_t gt_b = 0, eq_b = 0;
     for (int r = 0; r < rank; ++r) {
-        const uint32_t *rc = cluster.map_shared_rank(&s_cnt[0], r);
+        const uint32_t *rc = remote(&s_cnt[0], r);
         gt_b += rc[0];
         eq_b += rc[1];
     }
@@ -195,13 +242,29 @@ select_cluster_kernel(CacheView c, int src, const float *scores, int64_t score_s
         }
     }
     // No CTA may leave while another still reads its shared memory.
-    cluster.sync();
+    csync();
+}
+
+#define CSA2_SELECT_ARGS                                                                                      \
+    CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,               \
+        const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool, int32_t *pool_len
+#define CSA2_SELECT_PASS c, src, scores, score_stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len
+
+__global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREADS, 1)
+select_cluster_kernel(CSA2_SELECT_ARGS)
+{
+    select_body<SEL_CLUSTER>(CSA2_SELECT_PASS);
+}
+
+__global__ void __launch_bounds__(SEL_THREADS, 1) select_cta_kernel(CSA2_SELECT_ARGS)
+{
+    select_body<1>(CSA2_SELECT_PASS);
 }
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
-                          int32_t *pool_len, cudaStream_t st)
+                          int32_t *pool_len, int max_n, cudaStream_t st)
 {
     static bool attr_done[64] = {};
     int dev = 0;
@@ -210,14 +273,17 @@ cudaError_t launch_select(const CacheView &c, int src, const float *scores, int6
     const int smem = SEL_CAP * (int)sizeof(uint32_t);
     if (dev >= 64 || !attr_done[dev]) {
         e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done[dev] = true;
     }
     LaunchScope scope(CSA2_KERNEL_SELECT, st);
-    dim3 grid(SEL_CLUSTER, c.batch);
-    select_cluster_kernel<<<grid, SEL_THREADS, smem, st>>>(c, src, scores, stride, pool_len_in, ids, k, out,
-                                                           out_stride, expand, pool, pool_len);
-    return cudaGetLastError();
+    if (max_n <= SEL_CAP)   // fits one CTA's shared memory: no cluster barriers on the path
+        return launch_pdl(select_cta_kernel, dim3(1, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores, stride,
+                          pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
+    return launch_pdl(select_cluster_kernel, dim3(SEL_CLUSTER, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores,
+                      stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
 }
 
 }  // namespace csa2

@@ -9,7 +9,7 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
                          const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st);
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
-                          int32_t *pool_len, cudaStream_t st);
+                          int32_t *pool_len, int max_n, cudaStream_t st);
 cudaError_t launch_prefill(const CacheView &c, int req, int m, int tok_begin, int n_tok, int n_tok_final,
                            const float *lat, const float *key, const float *gate, cudaStream_t st);
 cudaError_t launch_append(const CacheView &c, const float *lat, const float *key, const float *gate,
@@ -18,7 +18,7 @@ cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, cons
                           void *out, int out_is_fp32, float *part_o, float *part_ml, cudaStream_t st);
 
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                               float *part_o, float *part_ml, cudaStream_t st);
+                               void *out, int out_is_fp32, float *part_o, cudaStream_t st);
 
 constexpr int ATT_KEYS_PER_SPLIT = 128;
 constexpr int ATT_SPLITS = (CSA2_TOPK + CSA2_SWA) / ATT_KEYS_PER_SPLIT;   // 5: four top-k tiles + the window

@@ -4,18 +4,23 @@
 // FP8 keys (FULL / REINDEX rescoring).  Source: 0539edu.com/news/5732216 §3
 // (indexer: 32 query heads x 128 dims; hierarchical blocks of 8 positions).
 //
-// Design (one persistent CTA per SM, 6 warps):
-//   warp 4      TMA producer: 128-row tiles (16 KB of FP8) into a 6-stage
+// Design (two persistent CTAs per SM, 6 warps each):
+//   warp 4      TMA producer: 128-row tiles (16 KB of FP8) into a 5-stage
 //               shared-memory ring, 128-byte swizzled, one box per page run.
-//   warps 0-3   thread = row: FP8 -> f16 (exact) straight into tensor memory
-//               as the MMA's A operand; then the epilogue reads the 32 head
-//               dot products of its row back from tensor memory and applies
-//               ReLU and the head weights.
-//   warp 5      allocates tensor memory and issues the MMAs:
-//               D[128 x 32] (fp32) = A[128 x 128] (f16, TMEM) . Q^T (f16, smem).
-// The query is converted once per request to f16 with an exact per-head
-// power-of-two scale (so every bf16 query value stays exact), undone on the
-// head weight: w_h * ReLU(dot) = (w_h * 2^-s) * ReLU(2^s dot).
+//   warp 5      allocates tensor memory and issues the MMAs straight on the
+//               FP8 tile: D[128 x 96] (fp32) = K[128 x 128] (e4m3) . Qs^T,
+//               kind::f8f6f4, where Qs stacks three e5m2 parts of the query
+//               (32 heads each); their sum is the query exactly (see below).
+//   warps 0-3   convert the query once per request; thread = row epilogue:
+//               dot_h = D[h] + D[32+h] + D[64+h], score = sum_h w'_h ReLU(dot_h).
+// Query split: per head, q' = q * 2^s with max|q'| in [2^14, 2^15); then
+// q' = p1 + p2 + p3 with p1 = e5m2(q'), p2 = e5m2(q' - p1), p3 = e5m2(rest).
+// A bf16 value has 8 significant bits and each e5m2 part takes 3, so the sum
+// is exact for every element not below 2^-9 (e5m2 steps of 2^-16), i.e. down
+// to 2^-24 of the head's largest entry; w'_h = w_h * 2^-s undoes the scale.
+// The tensor cores accumulate these products at fp32 precision (checked on
+// hardware against exact sums), so the scores are fp32-accumulated
+// sum_h w_h ReLU(q_h . k) as the method defines them.
 // Tiles of all requests form one list split evenly over the CTAs.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -30,14 +35,25 @@ using namespace umma;
 namespace {
 
 constexpr int TILE = 128;
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
+constexpr int CTAS_PER_SM = 2;                              // two independent pipelines per SM
+constexpr int PW = 16;                                      // producer look-up window (tiles)
 constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;            // 16 KB
-constexpr int QBYTES = CSA2_IDX_HEADS * CSA2_KEY_DIM * 2;   // 8 KB of f16
+constexpr int QPARTS = 3;
+constexpr int QROWS = QPARTS * CSA2_IDX_HEADS;              // 96 = MMA N
+constexpr int QBYTES = QROWS * CSA2_KEY_DIM;                // 12 KB of e5m2
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t A_COL0 = 0, D_COL0 = 128;                // A: 2 x 64 cols, D: 2 x 32 cols
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 2 * QBYTES;
-constexpr uint32_t IDESC = idesc_f16(128, 32, false, false, false);
+constexpr uint32_t TMEM_COLS = 256;                         // D: 2 x 96 columns
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + QBYTES;   // + 8 * (batch + 1)
+constexpr int MAX_BATCH = 1024;
+// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, N = 96, M = 128.
+constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(QROWS >> 3) << 17) | (8u << 24);
+
+// 2-D views (rows of 128 bytes) of the summary and key planes, with boxes of
+// one 8-row run, one 64-row page and one whole 128-row tile.
+struct PlaneMaps {
+    CUtensorMap summ8, summ128, keys8, keys64, keys128;
+};
 
 struct Params {
     CacheView c;
@@ -58,23 +74,30 @@ __device__ __forceinline__ int rows_of_req(const Params &p, int b)
     return max(0, min(p.pool_len[b], CSA2_POOL));
 }
 
-// Walks this CTA's contiguous slice [i0, i1) of the global tile list.
+// Walks this CTA's contiguous slice [i0, i1) of the global tile list, using
+// the per-request row counts and tile prefix sums kept in shared memory.
 struct TileIter {
     int b, t, rows, tiles, left;
-    __device__ void init(const Params &p, long long i0, long long i1)
+    const int *s_rows, *s_pre;   // s_pre[b] = tiles of requests < b; s_pre[batch] = total
+    int batch;
+    __device__ void init(const int *rows_, const int *pre_, int batch_, long long i0, long long i1)
     {
+        s_rows = rows_;
+        s_pre = pre_;
+        batch = batch_;
         left = (int)(i1 - i0);
-        b = 0;
-        long long acc = 0;
-        for (; b < p.c.batch; ++b) {
-            rows = rows_of_req(p, b);
-            tiles = (rows + TILE - 1) / TILE;
-            if (i0 < acc + tiles) break;
-            acc += tiles;
+        int lo = 0, hi = batch;                      // last b with s_pre[b] <= i0 and tiles > 0
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_pre[mid] <= i0) lo = mid; else hi = mid;
         }
-        t = (int)(i0 - acc);
+        b = lo;
+        while (b < batch - 1 && s_pre[b + 1] <= i0) ++b;
+        rows = s_rows[b];
+        tiles = s_pre[b + 1] - s_pre[b];
+        t = (int)(i0 - s_pre[b]);
     }
-    __device__ void next(const Params &p)
+    __device__ void next()
     {
         --left;
         if (left <= 0) return;
@@ -82,8 +105,8 @@ struct TileIter {
         while (t >= tiles) {
             ++b;
             t = 0;
-            rows = rows_of_req(p, b);
-            tiles = (rows + TILE - 1) / TILE;
+            rows = s_rows[b];
+            tiles = s_pre[b + 1] - s_pre[b];
         }
     }
 };
@@ -101,40 +124,74 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 
 __device__ __forceinline__ void bar_workers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__global__ void __launch_bounds__(THREADS, 1)
-score_umma_kernel(const __grid_constant__ CUtensorMap map_summ, const __grid_constant__ CUtensorMap map_keys64,
-                  const __grid_constant__ CUtensorMap map_keys8, Params p)
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile("{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+                 : "memory");
+}
+
+__device__ __forceinline__ float e5m2_to_f32(uint8_t c)
+{
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E5M2);
+    return __half2float(__half(h));
+}
+
+__global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
+score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *qbuf = sm + STAGES * STAGE_BYTES;
-    __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], a_full[2], d_full[2], d_empty[2];
-    __shared__ float wq[2][CSA2_IDX_HEADS];
+    __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], d_full[2], d_empty[2], q_full;
+    __shared__ float wq[CSA2_IDX_HEADS];
     __shared__ uint32_t tmem_base;
     __shared__ long long s_total;
     __shared__ volatile int s_abort;
+    __shared__ int win_b[2][PW], win_r0[2][PW], win_n[2][PW], win_pid[2][PW][16];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (warp == 5) tmem_alloc(&tmem_base, TMEM_COLS);
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 4);
+            mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&a_full[i], 4);
             mbar_init(&d_full[i], 1);
             mbar_init(&d_empty[i], 4);
         }
+        mbar_init(&q_full, 1);
         s_abort = 0;
         mbar_fence_init();
     }
+    int *s_rows = reinterpret_cast<int *>(qbuf + QBYTES), *s_pre = s_rows + p.c.batch;
+    grid_dependency_wait();                      // inputs may come from the previous kernel
+    allow_dependents();
     if (warp == 0) {
-        long long tot = 0;
-        for (int b = lane; b < p.c.batch; b += 32) tot += (rows_of_req(p, b) + TILE - 1) / TILE;
+        // rows and tile prefix sums of every request, 32 requests per round
+        int carry = 0;
+        for (int b0 = 0; b0 < p.c.batch; b0 += 32) {
+            const int b = b0 + lane;
+            const int rows = b < p.c.batch ? rows_of_req(p, b) : 0;
+            const int tiles = (rows + TILE - 1) / TILE;
+            int incl = tiles;
 #pragma unroll
-        for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-        if (lane == 0) s_total = tot;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (b < p.c.batch) {
+                s_rows[b] = rows;
+                s_pre[b] = carry + incl - tiles;
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            s_pre[p.c.batch] = carry;
+            s_total = carry;
+        }
     }
     __syncthreads();
     fence_after_sync();
@@ -146,61 +203,126 @@ score_umma_kernel(const __grid_constant__ CUtensorMap map_summ, const __grid_con
 
     if (warp == 4 && n_items > 0) {
         // ------------------------------------------------------------ producer
+        // Page ids are looked up a window of PW tiles at a time, all lanes in
+        // parallel, so the issue loop never waits on a dependent global load.
+        const int chunk_rows = (p.src == ROWS_KEYS) ? 64 : 8;
+        const int full_chunks = TILE / chunk_rows;                  // chunks of a complete tile
+        const uint32_t chunk_bytes = (uint32_t)chunk_rows * CSA2_KEY_DIM;
+        const int rows_per_page = (p.src == ROWS_SUMMARIES) ? 8 : 64;
+        const CUtensorMap *m_chunk = (p.src == ROWS_SUMMARIES) ? &maps.summ8 : (p.src == ROWS_KEYS) ? &maps.keys64
+                                                                                                  : &maps.keys8;
+        const CUtensorMap *m_tile = (p.src == ROWS_SUMMARIES) ? &maps.summ128 : &maps.keys128;
         if (lane == 0) {
-            tma_prefetch_map(&map_summ);
-            tma_prefetch_map(&map_keys64);
-            tma_prefetch_map(&map_keys8);
+            tma_prefetch_map(m_chunk);
+            tma_prefetch_map(m_tile);
         }
         TileIter it;
-        it.init(p, i0, i1);
+        it.init(s_rows, s_pre, p.c.batch, i0, i1);
         int issued = 0;
-        for (int j = 0; j < n_items; ++j, it.next(p)) {
-            const int s = j % STAGES;
-            if (j >= STAGES && !wait_or_abort(&empty[s], ((j / STAGES) - 1) & 1, abort, p.c.error)) break;
-            const int b = it.b, r0 = it.t * TILE;
-            const int valid = min(TILE, it.rows - r0);
-            // Lane l prepares chunk l of this tile (a page or an 8-row run).
-            int chunk_rows = (p.src == ROWS_KEYS) ? 64 : 8;
-            int n_chunks = (valid + chunk_rows - 1) / chunk_rows;
-            int pid = -1, y = 0;
-            if (lane < n_chunks) {
-                int e;                                   // first entry of the chunk
-                if (p.src == ROWS_SUMMARIES) e = (r0 + 8 * lane) * CSA2_BLOCK;
-                else if (p.src == ROWS_KEYS) e = r0 + 64 * lane;
-                else {
-                    e = p.pool[(size_t)b * CSA2_POOL + r0 + 8 * lane];
-                    if (e < 0 || e >= n_entries_of(p.c, b) || (e & 7)) {
-                        set_error(p.c.error, CSA2_DEV_BAD_INDEX);
-                        e = -1;
-                    }
+        bool stop = false;
+        const int n_win = (n_items + PW - 1) / PW;
+        // Window w's look-ups go to buffer w & 1.  The page-table loads of
+        // window w + 1 are issued before window w's copies and consumed after
+        // them, so their latency hides behind the copies.
+        int e_[8], b_[8], pg_[8];
+        auto meta = [&](int w) {                    // lane 0: tiles of window w
+            const int wb = w & 1, nw = min(PW, n_items - w * PW);
+            if (lane == 0)
+                for (int i = 0; i < nw; ++i, it.next()) {
+                    win_b[wb][i] = it.b;
+                    win_r0[wb][i] = it.t * TILE;
+                    win_n[wb][i] = (min(TILE, it.rows - it.t * TILE) + chunk_rows - 1) / chunk_rows;
                 }
-                if (e >= 0) {
-                    int pi = e >> 6;
-                    if (pi < p.c.max_pages) {
-                        int id = p.c.page_table[(size_t)b * p.c.max_pages + pi];
-                        if (id >= 0 && id < p.c.n_pages) {
-                            pid = id;
-                            y = (p.src == ROWS_SUMMARIES) ? 0 : (e & 63);
-                        } else {
-                            set_error(p.c.error, CSA2_DEV_BAD_PAGE);
-                        }
-                    } else {
-                        set_error(p.c.error, CSA2_DEV_CAPACITY);
-                    }
-                }
-            }
-            const uint32_t ok = __ballot_sync(0xffffffffu, pid >= 0);
-            const uint32_t chunk_bytes = (p.src == ROWS_KEYS) ? 8192u : 1024u;
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], __popc(ok) * chunk_bytes);
             __syncwarp();
-            if (pid >= 0) {
-                uint8_t *dst = sm + s * STAGE_BYTES + lane * chunk_bytes;
-                const CUtensorMap *m = (p.src == ROWS_SUMMARIES) ? &map_summ
-                                     : (p.src == ROWS_KEYS)      ? &map_keys64
-                                                                 : &map_keys8;
-                tma_load_3d(dst, m, 0, y, pid, &full[s]);
+        };
+        auto issue_loads = [&](int w) {             // non-blocking: loads in flight
+            const int wb = w & 1, nw = min(PW, n_items - w * PW);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int k = lane + 32 * u, i = k >> 4, ch = k & 15;
+                e_[u] = -1;
+                b_[u] = 0;
+                pg_[u] = -1;
+                if (i < nw && ch < win_n[wb][i]) {
+                    const int b = win_b[wb][i], r0 = win_r0[wb][i];
+                    b_[u] = b;
+                    if (p.src == ROWS_SUMMARIES) e_[u] = (r0 + 8 * ch) * CSA2_BLOCK;
+                    else if (p.src == ROWS_KEYS) e_[u] = r0 + 64 * ch;
+                    else e_[u] = p.pool[(size_t)b * CSA2_POOL + r0 + 8 * ch];
+                    if (p.src != ROWS_POOL && (e_[u] >> 6) < p.c.max_pages)
+                        pg_[u] = p.c.page_table[(size_t)b * p.c.max_pages + (e_[u] >> 6)];
+                }
             }
-            issued = j + 1;
+        };
+        auto finish = [&](int w) {                  // blocking: checks, then shared memory
+            const int wb = w & 1, nw = min(PW, n_items - w * PW);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int k = lane + 32 * u, i = k >> 4, ch = k & 15;
+                if (i >= nw) continue;
+                int pid = -1;
+                if (ch < win_n[wb][i]) {
+                    int e = e_[u], pg = pg_[u];
+                    if (p.src == ROWS_POOL) {
+                        if (e < 0 || e >= n_entries_of(p.c, b_[u]) || (e & 7)) {
+                            set_error(p.c.error, CSA2_DEV_BAD_INDEX);
+                            e = -1;
+                        } else if ((e >> 6) < p.c.max_pages) {
+                            pg = p.c.page_table[(size_t)b_[u] * p.c.max_pages + (e >> 6)];
+                        }
+                    }
+                    if (e >= 0) {
+                        if ((e >> 6) >= p.c.max_pages) {
+                            set_error(p.c.error, CSA2_DEV_CAPACITY);
+                        } else if (pg < 0 || pg >= p.c.n_pages) {
+                            set_error(p.c.error, CSA2_DEV_BAD_PAGE);
+                        } else {
+                            pid = pg * rows_per_page + ((p.src == ROWS_SUMMARIES) ? 0 : (e & 63));   // plane row
+                        }
+                    }
+                }
+                win_pid[wb][i][ch] = pid;
+            }
+            __syncwarp();
+        };
+        meta(0);
+        issue_loads(0);
+        finish(0);
+        for (int w = 0; w < n_win && !stop; ++w) {
+            const int wb = w & 1, nw = min(PW, n_items - w * PW);
+            if (w + 1 < n_win) {
+                meta(w + 1);
+                issue_loads(w + 1);
+            }
+            for (int i = 0; i < nw; ++i) {
+                const int j = w * PW + i, s = j % STAGES;
+                bool okw = true;
+                if (lane == 0 && j >= STAGES) okw = wait_or_abort(&empty[s], ((j / STAGES) - 1) & 1, abort, p.c.error);
+                if (!__shfl_sync(0xffffffffu, okw, 0)) {          // warp-uniform decision
+                    stop = true;
+                    break;
+                }
+                const int row = lane < 16 ? win_pid[wb][i][lane] : -1;       // first plane row of the chunk
+                const uint32_t ok = __ballot_sync(0xffffffffu, row >= 0);
+                const int row0 = __shfl_sync(0xffffffffu, row, 0);
+                const bool contig = __popc(ok) == full_chunks &&
+                                    __all_sync(0xffffffffu, lane >= full_chunks || row == row0 + lane * chunk_rows);
+                uint8_t *dst = sm + s * STAGE_BYTES;
+                if (contig) {
+                    // the whole tile is one run of plane rows: a single 16 KB copy
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                        tma_load_2d(dst, m_tile, 0, row0, &full[s]);
+                    }
+                } else {
+                    if (lane == 0) mbar_arrive_expect_tx(&full[s], __popc(ok) * chunk_bytes);
+                    __syncwarp();
+                    if (row >= 0) tma_load_2d(dst + lane * chunk_bytes, m_chunk, 0, row, &full[s]);
+                }
+                __syncwarp();
+                issued = j + 1;
+            }
+            if (!stop && w + 1 < n_win) finish(w + 1);
         }
         // Never leave with copies in flight: wait for the last stages to land.
         if (lane == 0)
@@ -209,25 +331,31 @@ score_umma_kernel(const __grid_constant__ CUtensorMap map_summ, const __grid_con
     } else if (warp == 5 && n_items > 0) {
         // ------------------------------------------------------------ MMA issuer
         TileIter it;
-        it.init(p, i0, i1);
+        it.init(s_rows, s_pre, p.c.batch, i0, i1);
         int cur_b = -1, sw = -1, issued = 0;
-        for (int j = 0; j < n_items; ++j, it.next(p)) {
+        const uint32_t qaddr = smem_addr(qbuf);
+        for (int j = 0; j < n_items; ++j, it.next()) {
+            const int ab = j & 1, s = j % STAGES;
+            bool okw = true;
+            if (lane == 0) {
+                if (it.b != cur_b) okw = wait_or_abort(&q_full, (sw + 1) & 1, abort, p.c.error);
+                if (okw) okw = wait_or_abort(&full[s], (j / STAGES) & 1, abort, p.c.error);
+                if (okw && j >= 2) okw = wait_or_abort(&d_empty[ab], ((j >> 1) - 1) & 1, abort, p.c.error);
+            }
             if (it.b != cur_b) {
                 cur_b = it.b;
                 ++sw;
             }
-            const int ab = j & 1, qb = sw & 1;
-            if (!wait_or_abort(&a_full[ab], (j >> 1) & 1, abort, p.c.error)) break;
-            if (j >= 2 && !wait_or_abort(&d_empty[ab], ((j >> 1) - 1) & 1, abort, p.c.error)) break;
+            if (!__shfl_sync(0xffffffffu, okw, 0)) break;          // warp-uniform decision
             fence_after_sync();
             if (lane == 0) {
-                const uint32_t qaddr = smem_addr(qbuf + qb * QBYTES);
+                const uint32_t aaddr = smem_addr(sm + s * STAGE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < CSA2_KEY_DIM / 16; ++kk) {
-                    uint64_t bd = smem_desc(qaddr + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024);
-                    mma_ts(tb + D_COL0 + 32 * ab, tb + A_COL0 + 64 * ab + 8 * kk, bd, IDESC, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < CSA2_KEY_DIM / 32; ++kk)
+                    mma_f8(tb + QROWS * ab, smem_desc(aaddr + kk * 32, 16, 1024), smem_desc(qaddr + kk * 32, 16, 1024),
+                           IDESC, kk > 0 ? 1u : 0u);
                 mma_commit(&d_full[ab]);
+                mma_commit(&empty[s]);                              // stage free once the MMAs have read it
             }
             __syncwarp();
             issued = j + 1;
@@ -238,32 +366,14 @@ score_umma_kernel(const __grid_constant__ CUtensorMap map_summ, const __grid_con
     } else if (warp < 4 && n_items > 0) {
         // ------------------------------------------------------------ workers
         TileIter it;
-        it.init(p, i0, i1);
+        it.init(s_rows, s_pre, p.c.batch, i0, i1);
         const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        int cur_b = -1, sw = -1;
-        int pb = 0, pt = 0, prow = 0, pqb = 0;       // previous item (for its epilogue)
-        auto epilogue = [&](int i, int b, int t, int rows, int qb) {
-            const int db = i & 1;
-            bool ok = wait_or_abort(&d_full[db], (i >> 1) & 1, abort, p.c.error);
-            fence_after_sync();
-            uint32_t r[32];
-            tmem_ld32(tb + lane_base + D_COL0 + 32 * db, r);
-            tmem_ld_wait();
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&d_empty[db]);
-            float sc = 0.0f;
-#pragma unroll
-            for (int h = 0; h < CSA2_IDX_HEADS; ++h) sc = fmaf(wq[qb][h], fmaxf(__uint_as_float(r[h]), 0.0f), sc);
-            const int row = t * TILE + tid;
-            if (ok && row < rows) p.scores[(size_t)b * p.stride + row] = sc;
-        };
-        for (int j = 0; j < n_items; ++j, it.next(p)) {
+        int cur_b = -1;
+        for (int j = 0; j < n_items; ++j, it.next()) {
             if (it.b != cur_b) {
-                // New request: convert its query into the free q buffer.
+                // New request.  Every MMA issued so far has completed (the
+                // previous epilogue waited for it), so the q buffer is free.
                 cur_b = it.b;
-                ++sw;
-                const int qb = sw & 1;
                 const int h = tid >> 2, qd = tid & 3;
                 const uint4 *src = reinterpret_cast<const uint4 *>(p.q_idx + ((size_t)cur_b * CSA2_IDX_HEADS + h) *
                                                                                  CSA2_KEY_DIM + 32 * qd);
@@ -271,71 +381,78 @@ score_umma_kernel(const __grid_constant__ CUtensorMap map_summ, const __grid_con
 #pragma unroll
                 for (int i = 0; i < 4; ++i) raw[i] = src[i];
                 const uint32_t *rw = reinterpret_cast<const uint32_t *>(raw);
+                float x[32];
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    amax = fmaxf(amax, fabsf(__uint_as_float(rw[i] << 16)));
-                    amax = fmaxf(amax, fabsf(__uint_as_float(rw[i] & 0xffff0000u)));
+                    x[2 * i] = __uint_as_float(rw[i] << 16);
+                    x[2 * i + 1] = __uint_as_float(rw[i] & 0xffff0000u);
+                    amax = fmaxf(amax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
                 }
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
                 int ex = 0;
                 if (amax > 0.0f) frexpf(amax, &ex);
                 const int sh = (amax > 0.0f) ? 15 - ex : 0;          // amax * 2^sh in [2^14, 2^15)
-                uint8_t *qdst = qbuf + qb * QBYTES + (qd >> 1) * 4096 + h * 128;
+                uint32_t part[QPARTS][8];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t o[4];
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t w0 = 0, w1 = 0, w2 = 0;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint32_t v = rw[4 * cc + i];
-                        __half lo = __float2half_rn(ldexpf(__uint_as_float(v << 16), sh));
-                        __half hi = __float2half_rn(ldexpf(__uint_as_float(v & 0xffff0000u), sh));
-                        o[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+                    for (int k = 0; k < 4; ++k) {
+                        float r = ldexpf(x[4 * i + k], sh);
+                        const uint8_t c0 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
+                        r -= e5m2_to_f32(c0);
+                        const uint8_t c1 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
+                        r -= e5m2_to_f32(c1);
+                        const uint8_t c2 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
+                        w0 |= (uint32_t)c0 << (8 * k);
+                        w1 |= (uint32_t)c1 << (8 * k);
+                        w2 |= (uint32_t)c2 << (8 * k);
                     }
-                    const int chunk = 4 * (qd & 1) + cc;
-                    *reinterpret_cast<uint4 *>(qdst + ((chunk ^ (h & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    part[0][i] = w0;
+                    part[1][i] = w1;
+                    part[2][i] = w2;
                 }
-                if (qd == 0) wq[qb][h] = ldexpf(p.w[(size_t)cur_b * CSA2_IDX_HEADS + h], -sh);
+                // row n = part * 32 + h, bytes 32*qd .. +31 = 16-byte chunks 2qd, 2qd+1
+#pragma unroll
+                for (int pp = 0; pp < QPARTS; ++pp) {
+                    const int n = pp * CSA2_IDX_HEADS + h;
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int chunk = 2 * qd + cc;
+                        *reinterpret_cast<uint4 *>(qbuf + n * 128 + ((chunk ^ (n & 7)) << 4)) =
+                            make_uint4(part[pp][4 * cc], part[pp][4 * cc + 1], part[pp][4 * cc + 2],
+                                       part[pp][4 * cc + 3]);
+                    }
+                }
+                if (qd == 0) wq[h] = ldexpf(p.w[(size_t)cur_b * CSA2_IDX_HEADS + h], -sh);
                 fence_proxy_async_smem();
                 bar_workers();
+                if (tid == 0) mbar_arrive(&q_full);
             }
-            const int s = j % STAGES, ab = j & 1;
-            wait_or_abort(&full[s], (j / STAGES) & 1, abort, p.c.error);
-            // Row tid of the tile: 8 swizzled 16-byte chunks -> 64 f16x2 columns.
-            const uint8_t *row = sm + s * STAGE_BYTES + tid * 128;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t cols[32];
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int c = 4 * half + c4;
-                    uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (tid & 7)) << 4));
-                    uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(wv[i] & 0xffff), __NV_E4M3);
-                        __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(wv[i] >> 16), __NV_E4M3);
-                        cols[8 * c4 + 2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-                        cols[8 * c4 + 2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
-                    }
-                }
-                tmem_st32(tb + lane_base + A_COL0 + 64 * ab + 32 * half, cols);
-            }
-            tmem_st_wait();
+            // ---- epilogue of tile j
+            const int db = j & 1;
+            const bool ok = wait_or_abort(&d_full[db], (j >> 1) & 1, abort, p.c.error);
+            fence_after_sync();
+            uint32_t r0[32], r1[32], r2[32];
+            tmem_ld32(tb + lane_base + QROWS * db, r0);
+            tmem_ld32(tb + lane_base + QROWS * db + 32, r1);
+            tmem_ld32(tb + lane_base + QROWS * db + 64, r2);
+            tmem_ld_wait();
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&a_full[ab]);
-                mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&d_empty[db]);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int hh = 0; hh < CSA2_IDX_HEADS; ++hh) {
+                const float dot = (__uint_as_float(r0[hh]) + __uint_as_float(r1[hh])) + __uint_as_float(r2[hh]);
+                acc[hh & 3] = fmaf(wq[hh], fmaxf(dot, 0.0f), acc[hh & 3]);
             }
-            if (j > 0) epilogue(j - 1, pb, pt, prow, pqb);
-            pb = it.b;
-            pt = it.t;
-            prow = it.rows;
-            pqb = sw & 1;
+            const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            const int row = it.t * TILE + tid;
+            if (ok && row < it.rows) p.scores[(size_t)it.b * p.stride + row] = sc;
         }
-        epilogue(n_items - 1, pb, pt, prow, pqb);
     }
     fence_before_sync();
     __syncthreads();
@@ -346,29 +463,17 @@ score_umma_kernel(const __grid_constant__ CUtensorMap map_summ, const __grid_con
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+// 2-D byte tensor over a plane: rows of 128 bytes, boxes of box_rows rows,
+// 128-byte swizzled.
+bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows)
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
-    }
-    return fn;
-}
-
-// 3-D byte tensor over one page field: (128 bytes, slots, pages).
-bool make_page_map(CUtensorMap *m, void *base, int slots, int box_slots, int n_pages)
-{
-    auto fn = encode_fn();
+    auto fn = tensor_map_encoder();
     if (!fn) return false;
-    cuuint64_t dims[3] = {128, (cuuint64_t)slots, (cuuint64_t)n_pages};
-    cuuint64_t strides[2] = {128, CSA2_PAGE_BYTES};
-    cuuint32_t box[3] = {128, (cuuint32_t)box_slots, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -393,26 +498,29 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
                          const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st)
 {
     (void)max_rows;
+    if (c.batch > MAX_BATCH) return cudaErrorInvalidValue;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(score_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        e = cudaFuncSetAttribute(score_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(SMEM_BYTES + 8 * (MAX_BATCH + 1)));
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done[dev] = true;
     }
-    CUtensorMap m_summ, m_keys64, m_keys8;
-    if (!make_page_map(&m_summ, c.pool + CSA2_PAGE_SUMM_OFF, 8, 8, c.n_pages) ||
-        !make_page_map(&m_keys64, c.pool + CSA2_PAGE_KEYS_OFF, 64, 64, c.n_pages) ||
-        !make_page_map(&m_keys8, c.pool + CSA2_PAGE_KEYS_OFF, 64, 8, c.n_pages))
+    PlaneMaps maps;
+    const long long np = c.n_pages;
+    if (!make_plane_map(&maps.summ8, c.summ, np * 8, 8) || !make_plane_map(&maps.summ128, c.summ, np * 8, 128) ||
+        !make_plane_map(&maps.keys8, c.keys, np * 64, 8) || !make_plane_map(&maps.keys64, c.keys, np * 64, 64) ||
+        !make_plane_map(&maps.keys128, c.keys, np * 64, 128))
         return cudaErrorInvalidValue;
     Params p{c, src, q_idx, w, pool, pool_len, scores, stride};
     int kid = src == ROWS_KEYS ? CSA2_KERNEL_FLAT_SCORE : src == ROWS_SUMMARIES ? CSA2_KERNEL_BLOCK_SCORE
                                                                                 : CSA2_KERNEL_POOL_SCORE;
+    const size_t smem = SMEM_BYTES + 8 * ((size_t)c.batch + 1);
     LaunchScope scope(kid, st);
-    score_umma_kernel<<<sm_count(), THREADS, SMEM_BYTES, st>>>(m_summ, m_keys64, m_keys8, p);
-    return cudaGetLastError();
+    return launch_pdl(score_umma_kernel, dim3(CTAS_PER_SM * sm_count()), dim3(THREADS), smem, st, maps, p);
 }
 
 }  // namespace csa2

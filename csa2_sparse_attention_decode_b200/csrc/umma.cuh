@@ -15,6 +15,8 @@
 //     32-bit column (lower K in the low half).
 #pragma once
 #include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace csa2 {
@@ -141,10 +143,33 @@ __device__ __forceinline__ void tma_load_3d(void *dst_smem, const CUtensorMap *m
                  "l"((uint64_t)map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
                  : "memory");
 }
+__device__ __forceinline__ void tma_load_2d(void *dst_smem, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+                 "[%4];" ::"r"(smem_addr(dst_smem)),
+                 "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_addr(bar))
+                 : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
 
 }  // namespace umma
+
+// Driver entry point of cuTensorMapEncodeTiled (looked up once, no link-time
+// dependency on the driver library).
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
+    }
+    return fn;
+}
+
 }  // namespace csa2

@@ -16,9 +16,9 @@ from typing import List, Optional
 import torch
 
 import synth
-from . import (INDEX_FLAT, INDEX_FULL, INDEX_REINDEX, PAGE_BYTES, PAGE_CODES_OFF, PAGE_ENTRIES, PAGE_KEYS_OFF,
-               PAGE_SCALES_OFF, PAGE_SUMM_OFF, POOL, SWA_CODES_OFF, SWA_SCALE_OFF, TOPK, Cache, csa2_append,
-               csa2_attend, csa2_index, csa2_prefill, workspace)
+from . import (INDEX_FLAT, INDEX_FULL, INDEX_REINDEX, PAGE_CODES_BYTES, PAGE_ENTRIES, PAGE_KEYS_BYTES,
+               PAGE_SCALES_BYTES, PAGE_SUMM_BYTES, POOL, SWA_CODES_OFF, SWA_SCALE_OFF, TOPK, Cache, csa2_append,
+               csa2_attend, csa2_index, csa2_prefill, plane_offsets, workspace)
 
 SOFTMAX_SCALE = 1.0 / math.sqrt(512.0)
 PREFILL_CHUNK = 65536
@@ -93,22 +93,23 @@ class DeviceWorkload:
     def entry_rows(self, b: int, entries: torch.Tensor):
         """Packed bytes of entries of request b: (codes [n,256], scales [n,32], keys [n,128]) on CPU."""
         e = entries.to(torch.int64).cpu()
-        pids = self.page_table[b].to(torch.int64)[e // PAGE_ENTRIES]
-        slot = e % PAGE_ENTRIES
-        base = (pids * PAGE_BYTES).to(self.device)
-        slot = slot.to(self.device)
+        pids = self.page_table[b].to(torch.int64)[e // PAGE_ENTRIES].to(self.device)
+        slot = (e % PAGE_ENTRIES).to(self.device)
         pool = self.cache.pool
+        planes = plane_offsets(self.cache.n_pages)
 
-        def gather(off, width):
-            idx = base[:, None] + off + slot[:, None] * width + torch.arange(width, device=self.device)[None, :]
+        def gather(plane, page_bytes, width):
+            base = planes[plane] + pids * page_bytes + slot * width
+            idx = base[:, None] + torch.arange(width, device=self.device)[None, :]
             return pool[idx].cpu()
 
-        return gather(PAGE_CODES_OFF, 256), gather(PAGE_SCALES_OFF, 32), gather(PAGE_KEYS_OFF, 128)
+        return (gather(0, PAGE_CODES_BYTES, 256), gather(1, PAGE_SCALES_BYTES, 32),
+                gather(2, PAGE_KEYS_BYTES, 128))
 
     def summary_rows(self, b: int, blocks: torch.Tensor) -> torch.Tensor:
         blk = blocks.to(torch.int64).cpu()
         pids = self.page_table[b].to(torch.int64)[(blk * 8) // PAGE_ENTRIES]
-        base = (pids * PAGE_BYTES + PAGE_SUMM_OFF + (blk % 8) * 128).to(self.device)
+        base = (plane_offsets(self.cache.n_pages)[3] + pids * PAGE_SUMM_BYTES + (blk % 8) * 128).to(self.device)
         idx = base[:, None] + torch.arange(128, device=self.device)[None, :]
         return self.cache.pool[idx].cpu()
 

@@ -59,24 +59,34 @@ typedef struct CUstream_st *csa2_stream_t;   /* == cudaStream_t */
 #define CSA2_SWA           128    /* swa_window_size                            */
 
 /* ---- cache layout -------------------------------------------------------
- * Global KV lives in one pool of fixed-size pages of 64 entries.  Entry e of
+ * Global KV lives in one pool of n_pages pages of 64 entries.  Entry e of
  * request b lives in page page_table[b * max_pages + (e >> 6)], slot e & 63.
- * Inside a page the fields are stored as separate arrays (each 256-byte
- * aligned within the page):
- *   codes     [64][256] u8   FP4 e2m1 codes; byte j = channel 2j (low nibble)
- *                            | channel 2j+1 (high nibble); bit 3 = sign
- *   scales    [64][32]  u8   e4m3 scale of channels 16i .. 16i+15
- *   keys      [64][128] u8   FP8 e4m3 indexer key
- *   summaries [8][128]  u8   FP8 e4m3 mean of the keys of block (e >> 3)
- * Per request, the SWA ring holds the last min(n_tokens, 128) raw tokens:
- *   codes [128][512] u8 e4m3, then scale [128] f32 (a power of two); token
- *   position t sits in slot t % 128.                                         */
+ * The pool is stored as four planes, one per field, each holding that field
+ * for every page in page-id order (so consecutive pages are contiguous within
+ * a plane, and a scan over consecutive pages is one sequential stream):
+ *   codes     plane at 0                : [n_pages][64][256] u8  FP4 e2m1
+ *             codes; byte j = channel 2j (low nibble) | channel 2j+1 (high
+ *             nibble); bit 3 of a nibble = sign
+ *   scales    plane at n_pages * 16384  : [n_pages][64][32]  u8  e4m3 scale
+ *             of channels 16i .. 16i+15
+ *   keys      plane at n_pages * 18432  : [n_pages][64][128] u8  FP8 e4m3
+ *             indexer key
+ *   summaries plane at n_pages * 26624  : [n_pages][8][128]  u8  FP8 e4m3
+ *             mean of the keys of block (e >> 3)
+ * Pool size: n_pages * CSA2_PAGE_BYTES.  The plane offsets are multiples of
+ * 256 bytes.  Per request, the SWA ring holds the last min(n_tokens, 128)
+ * raw tokens: codes [128][512] u8 e4m3, then scale [128] f32 (a power of
+ * two); token position t sits in slot t % 128.                               */
 #define CSA2_PAGE_ENTRIES      64
-#define CSA2_PAGE_CODES_OFF    0
-#define CSA2_PAGE_SCALES_OFF   16384
-#define CSA2_PAGE_KEYS_OFF     18432
-#define CSA2_PAGE_SUMM_OFF     26624
+#define CSA2_PAGE_CODES_BYTES  16384
+#define CSA2_PAGE_SCALES_BYTES 2048
+#define CSA2_PAGE_KEYS_BYTES   8192
+#define CSA2_PAGE_SUMM_BYTES   1024
 #define CSA2_PAGE_BYTES        27648
+#define CSA2_PLANE_CODES(n_pages)  ((size_t)0)
+#define CSA2_PLANE_SCALES(n_pages) ((size_t)(n_pages) * 16384)
+#define CSA2_PLANE_KEYS(n_pages)   ((size_t)(n_pages) * 18432)
+#define CSA2_PLANE_SUMM(n_pages)   ((size_t)(n_pages) * 26624)
 #define CSA2_SWA_CODES_OFF     0
 #define CSA2_SWA_SCALE_OFF     65536
 #define CSA2_SWA_BYTES         66048
