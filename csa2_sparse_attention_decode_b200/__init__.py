@@ -65,7 +65,7 @@ def _load():
         "csa2_prefill": (C.c_int, [P, I32, I32, I32, I32, I32, P, P, P, P]),
         "csa2_append": (C.c_int, [P, P, P, P, P, P]),
         "csa2_index": (C.c_int, [P, C.c_int, P, P, P, P, P, P, SZ, P]),
-        "csa2_attend": (C.c_int, [P, I32, P, P, C.c_float, P, I32, P, SZ, P]),
+        "csa2_attend": (C.c_int, [P, I32, P, P, C.c_float, P, I32, C.c_uint32, P, SZ, P]),
         "csa2_get_device_error": (C.c_int, [P, C.POINTER(C.c_int32), P]),
         "csa2_status_string": (C.c_char_p, [C.c_int]),
         "csa2_set_profile_events": (C.c_int, [I32, P, P]),
@@ -176,12 +176,15 @@ def csa2_index(cache: Cache, mode: int, q_idx, w, pool, pool_len, topk, ws, stre
                                         _ptr(topk), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def csa2_attend(cache: Cache, q, topk, scale: float, out, ws, stream=None):
+ATTEND_INPUTS_SETTLED = 1
+
+
+def csa2_attend(cache: Cache, q, topk, scale: float, out, ws, stream=None, flags: int = 0):
     heads = int(q.shape[1])
     qq = q.view(torch.int16) if q.dtype == torch.bfloat16 else q
     fp32 = 1 if out.dtype == torch.float32 else 0
     _check("csa2_attend", lib.csa2_attend(cache.ref, heads, _ptr(qq), _ptr(topk), float(scale), _ptr(out), fp32,
-                                          _ptr(ws), ws.numel(), _stream(stream)))
+                                          flags, _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def csa2_get_device_error(cache: Cache, stream=None) -> int:

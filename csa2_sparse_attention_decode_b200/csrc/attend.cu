@@ -13,10 +13,10 @@
 namespace csa2 {
 
 cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                          void *out, int out_is_fp32, float *part_o, float *part_ml, cudaStream_t st)
+                          void *out, int out_is_fp32, uint32_t flags, float *part_o, float *part_ml, cudaStream_t st)
 {
     (void)part_ml;
-    return launch_attend_umma(c, heads, q, topk, scale, out, out_is_fp32, part_o, st);
+    return launch_attend_umma(c, heads, q, topk, scale, out, out_is_fp32, flags, part_o, st);
 }
 
 }  // namespace csa2

@@ -70,7 +70,7 @@ extern "C" csa2_status csa2_attend_noalloc(const csa2_cache *cache, int32_t head
     // nothing left over from an earlier call needs clearing.
     float *part_o = scratch;
     float *part_ml = scratch + kPartO;
-    cudaError_t e = csa2::launch_attend(csa2::make_view(cache), heads, q, topk, scale, out, out_is_fp32, part_o,
+    cudaError_t e = csa2::launch_attend(csa2::make_view(cache), heads, q, topk, scale, out, out_is_fp32, 0u, part_o,
                                         part_ml, (cudaStream_t)stream);
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

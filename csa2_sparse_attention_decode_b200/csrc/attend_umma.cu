@@ -105,7 +105,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
 
 __global__ void __cluster_dims__(NTILES, 1, 1) __launch_bounds__(THREADS, 1)
 attend_umma_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads, const int32_t *topk, float scale,
-                   void *out, int out_is_fp32, float *part_o)
+                   void *out, int out_is_fp32, uint32_t flags, float *part_o)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -114,7 +114,7 @@ attend_umma_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int h
     __shared__ __align__(8) uint64_t bar_q, bar_s, bar_o;
     __shared__ uint32_t tmem_base;
     __shared__ float m_s[HG], l_s[HG], fac_s[HG], red_s[4][HG];
-    __shared__ int any_valid, tile_live[NTILES];
+    __shared__ int tile_live[NTILES];
     cg::cluster_group cluster = cg::this_cluster();
 
     const int tile = blockIdx.x, hg0 = blockIdx.y * HG, b = blockIdx.z;
@@ -122,13 +122,87 @@ attend_umma_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int h
     const int row = tid & (KT - 1), half = tid >> 7;      // two threads per key / tensor-memory row
     if (warp == 0) tmem_alloc(&tmem_base, TMEM_COLS);
     if (tid == 32) tma_prefetch_map(&map_q);
-    grid_dependency_wait();                               // q, top-k and the cache may be fresh
+    const bool early = (flags & CSA2_ATTEND_INPUTS_SETTLED) != 0;
+    bool valid = false;
+    // ---- 2. key `row`, channels [256*half, 256*half + 256) -> bf16 in slabs 4*half .. 4*half+3
+    auto gather = [&]() {
+        const int n_tok = c.n_tokens[b];
+        const int n_entries = n_entries_of(c, b);
+        const int nv = max(0, min(n_tok, CSA2_SWA));
+        if (tile < CSA2_TOPK / KT) {
+            const int e = topk[(size_t)b * CSA2_TOPK + tile * KT + row];
+            if (e >= n_entries && half == 0) set_error(c.error, CSA2_DEV_BAD_INDEX);
+            const int pid = (e >= 0 && e < n_entries) ? entry_pid(c, b, e) : -1;
+            if (pid >= 0) {
+                valid = true;
+                const int slot = e & (CSA2_PAGE_ENTRIES - 1);
+                const uint4 *codes = reinterpret_cast<const uint4 *>(codes_row(c, pid, slot)) + 8 * half;
+                const uint4 sv = reinterpret_cast<const uint4 *>(scales_row(c, pid, slot))[half];
+                uint4 cw[8];                               // 128 code bytes, loads issued together
+    #pragma unroll
+                for (int i = 0; i < 8; ++i) cw[i] = codes[i];
+                const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+    #pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const int slab = 4 * half + s4;
+                    const uint32_t cwu[8] = {cw[2 * s4].x,     cw[2 * s4].y,     cw[2 * s4].z,     cw[2 * s4].w,
+                                             cw[2 * s4 + 1].x, cw[2 * s4 + 1].y, cw[2 * s4 + 1].z, cw[2 * s4 + 1].w};
+    #pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {                                  // 8 channels per chunk
+                        uint32_t o[4];
+                        e2m1x8_to_bf16(cwu[ch], o);
+                        // channels slab*64 + ch*8 .. +7 share scale byte slab*4 + ch/2
+                        const int si = s4 * 4 + (ch >> 1);
+                        const float sf = e4m3_to_f32((uint8_t)(sw[si >> 2] >> (8 * (si & 3))));
+                        const uint32_t s2 = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(sf)) * 0x10001u;
+    #pragma unroll
+                        for (int i = 0; i < 4; ++i) o[i] = bf16x2_mul(o[i], s2);
+                        *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + ((ch ^ (row & 7)) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+        } else if (row < nv) {
+            valid = true;
+            const uint8_t *swa = swa_base(c, b);
+            const float sc = reinterpret_cast<const float *>(swa + CSA2_SWA_SCALE_OFF)[row];
+            const uint4 *codes = reinterpret_cast<const uint4 *>(swa + CSA2_SWA_CODES_OFF + row * CSA2_LATENT) + 16 * half;
+            uint4 cv[16];
+    #pragma unroll
+            for (int i = 0; i < 16; ++i) cv[i] = codes[i];
+    #pragma unroll
+            for (int k = 0; k < 16; ++k) {                                          // 16 codes -> 2 chunks
+                const int slab = 4 * half + (k >> 2), ch0 = 2 * (k & 3);
+                const uint32_t cw[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w};
+                uint32_t o[8];
+    #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] & 0xffff), __NV_E4M3);
+                    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] >> 16), __NV_E4M3);
+                    __nv_bfloat162 a = __floats2bfloat162_rn(__half2float(__ushort_as_half(lo.x)) * sc,
+                                                             __half2float(__ushort_as_half(lo.y)) * sc);
+                    __nv_bfloat162 bq = __floats2bfloat162_rn(__half2float(__ushort_as_half(hi.x)) * sc,
+                                                              __half2float(__ushort_as_half(hi.y)) * sc);
+                    o[2 * i] = *reinterpret_cast<uint32_t *>(&a);
+                    o[2 * i + 1] = *reinterpret_cast<uint32_t *>(&bq);
+                }
+                *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + ((ch0 ^ (row & 7)) << 4)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + (((ch0 + 1) ^ (row & 7)) << 4)) =
+                    make_uint4(o[4], o[5], o[6], o[7]);
+            }
+        }
+        if (!valid) {
+            for (int s4 = 0; s4 < 4; ++s4)
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4 *>(Vs + (4 * half + s4) * V_SLAB + row * 128 + (ch << 4)) =
+                        make_uint4(0, 0, 0, 0);
+        }
+    };
+    if (early) gather();                                  // inputs settled: overlap the previous kernel
+    grid_dependency_wait();                               // q (and, unless settled, the rest) may be fresh
     allow_dependents();
-    const int n_tok = c.n_tokens[b];
-    const int n_entries = n_entries_of(c, b);
-    const int nv = max(0, min(n_tok, CSA2_SWA));
     const int nh = min(HG, heads - hg0);
-
     if (tid == 0) {
         mbar_init(&bar_q, 1);
         mbar_init(&bar_s, 1);
@@ -139,87 +213,12 @@ attend_umma_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int h
         mbar_arrive_expect_tx(&bar_q, Q_BYTES);
         for (int slab = 0; slab < 8; ++slab) tma_load_3d(Qs + slab * Q_SLAB, &map_q, 64 * slab, hg0, b, &bar_q);
     }
-    if (tid == 1) any_valid = 0;
-    __syncthreads();
-
-    // ---- 2. key `row`, channels [256*half, 256*half + 256) -> bf16 in slabs 4*half .. 4*half+3
-    bool valid = false;
-    if (tile < CSA2_TOPK / KT) {
-        const int e = topk[(size_t)b * CSA2_TOPK + tile * KT + row];
-        if (e >= n_entries && half == 0) set_error(c.error, CSA2_DEV_BAD_INDEX);
-        const int pid = (e >= 0 && e < n_entries) ? entry_pid(c, b, e) : -1;
-        if (pid >= 0) {
-            valid = true;
-            const int slot = e & (CSA2_PAGE_ENTRIES - 1);
-            const uint4 *codes = reinterpret_cast<const uint4 *>(codes_row(c, pid, slot)) + 8 * half;
-            const uint4 sv = reinterpret_cast<const uint4 *>(scales_row(c, pid, slot))[half];
-            uint4 cw[8];                               // 128 code bytes, loads issued together
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cw[i] = codes[i];
-            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4) {
-                const int slab = 4 * half + s4;
-                const uint32_t cwu[8] = {cw[2 * s4].x,     cw[2 * s4].y,     cw[2 * s4].z,     cw[2 * s4].w,
-                                         cw[2 * s4 + 1].x, cw[2 * s4 + 1].y, cw[2 * s4 + 1].z, cw[2 * s4 + 1].w};
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {                                  // 8 channels per chunk
-                    uint32_t o[4];
-                    e2m1x8_to_bf16(cwu[ch], o);
-                    // channels slab*64 + ch*8 .. +7 share scale byte slab*4 + ch/2
-                    const int si = s4 * 4 + (ch >> 1);
-                    const float sf = e4m3_to_f32((uint8_t)(sw[si >> 2] >> (8 * (si & 3))));
-                    const uint32_t s2 = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(sf)) * 0x10001u;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) o[i] = bf16x2_mul(o[i], s2);
-                    *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + ((ch ^ (row & 7)) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            }
-        }
-    } else if (row < nv) {
-        valid = true;
-        const uint8_t *swa = swa_base(c, b);
-        const float sc = reinterpret_cast<const float *>(swa + CSA2_SWA_SCALE_OFF)[row];
-        const uint4 *codes = reinterpret_cast<const uint4 *>(swa + CSA2_SWA_CODES_OFF + row * CSA2_LATENT) + 16 * half;
-        uint4 cv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cv[i] = codes[i];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {                                          // 16 codes -> 2 chunks
-            const int slab = 4 * half + (k >> 2), ch0 = 2 * (k & 3);
-            const uint32_t cw[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w};
-            uint32_t o[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] & 0xffff), __NV_E4M3);
-                __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(cw[i] >> 16), __NV_E4M3);
-                __nv_bfloat162 a = __floats2bfloat162_rn(__half2float(__ushort_as_half(lo.x)) * sc,
-                                                         __half2float(__ushort_as_half(lo.y)) * sc);
-                __nv_bfloat162 bq = __floats2bfloat162_rn(__half2float(__ushort_as_half(hi.x)) * sc,
-                                                          __half2float(__ushort_as_half(hi.y)) * sc);
-                o[2 * i] = *reinterpret_cast<uint32_t *>(&a);
-                o[2 * i + 1] = *reinterpret_cast<uint32_t *>(&bq);
-            }
-            *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + ((ch0 ^ (row & 7)) << 4)) =
-                make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4 *>(Vs + slab * V_SLAB + row * 128 + (((ch0 + 1) ^ (row & 7)) << 4)) =
-                make_uint4(o[4], o[5], o[6], o[7]);
-        }
-    }
-    if (!valid) {
-        for (int s4 = 0; s4 < 4; ++s4)
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4 *>(Vs + (4 * half + s4) * V_SLAB + row * 128 + (ch << 4)) =
-                    make_uint4(0, 0, 0, 0);
-    }
-    if (valid) any_valid = 1;
+    if (!early) gather();
     fence_proxy_async_smem();
-    __syncthreads();
+    const bool live = __syncthreads_or(valid) != 0;      // any valid key in this tile
     fence_after_sync();
     const uint32_t tb = tmem_base;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const bool live = any_valid != 0;
 
     if (live) {
         // ---- 3. S^T = V . Q^T
@@ -406,7 +405,7 @@ bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch)
 }  // namespace
 
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                               void *out, int out_is_fp32, float *part_o, cudaStream_t st)
+                               void *out, int out_is_fp32, uint32_t flags, float *part_o, cudaStream_t st)
 {
     static bool attr_done[64] = {};
     int dev = 0;
@@ -422,7 +421,7 @@ cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q,
     dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);
     LaunchScope scope(CSA2_KERNEL_ATTEND, st);
     return launch_pdl(attend_umma_kernel, grid, dim3(THREADS), SMEM_BYTES, st, map_q, c, heads, topk, scale, out,
-                      out_is_fp32, part_o);
+                      out_is_fp32, flags, part_o);
 }
 
 }  // namespace csa2

@@ -154,7 +154,8 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
 }
 
 csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *q, const int32_t *topk, float scale,
-                        void *out, int32_t out_is_fp32, void *ws, size_t ws_bytes, csa2_stream_t stream)
+                        void *out, int32_t out_is_fp32, uint32_t flags, void *ws, size_t ws_bytes,
+                        csa2_stream_t stream)
 {
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
@@ -163,8 +164,9 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
     const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
     Workspace W = layout(ws, cache->batch, heads, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
-    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, W.part_o, W.part_ml,
-                                   (cudaStream_t)stream));
+    if (flags & ~CSA2_ATTEND_INPUTS_SETTLED) return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, flags, W.part_o,
+                                   W.part_ml, (cudaStream_t)stream));
 }
 
 csa2_status csa2_get_device_error(const csa2_cache *cache, int32_t *code_out, csa2_stream_t stream)

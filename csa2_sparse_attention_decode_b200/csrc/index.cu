@@ -26,6 +26,7 @@ __device__ __forceinline__ uint32_t ord_key(float x)
 constexpr int SEL_CLUSTER = 8;         // CTAs per request (one thread-block cluster)
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_CAP = 32768;         // keys a CTA keeps in shared memory (128 KB)
+constexpr int SEL_CAND = 2048;         // candidate keys kept after the first radix pass
 
 // Inclusive scan over threads 0..255 (warps 0..7); every thread of the CTA
 // must call it.  Returns the prefix for threads < 256.
@@ -98,6 +99,8 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     const float *s = scores + (size_t)b * score_stride + lo;
     auto key_at = [&](int e) -> uint32_t { return in_smem ? keys[e] : ord_key(s[e]); };
 
+    uint32_t *cand_key = keys + SEL_CAP, *cand_idx = cand_key + SEL_CAND;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
     if (in_smem) {
         // 8 independent loads in flight per thread per round.
         for (int e0 = 0; e0 < cnt; e0 += 8 * SEL_THREADS) {
@@ -110,34 +113,74 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int e = e0 + u * SEL_THREADS + tid;
-                if (e < cnt) keys[e] = ord_key(v[u]);
+                if (e < cnt) {
+                    const uint32_t key = ord_key(v[u]);
+                    keys[e] = key;
+                    kmin = min(kmin, key);
+                    kmax = max(kmax, key);
+                }
             }
+        }
+    } else {
+        for (int e = tid; e < cnt; e += SEL_THREADS) {
+            const uint32_t key = ord_key(s[e]);
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
         }
     }
     uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kk;
     if (!take_all) {
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass, buf = pass & 1;
-            // Per-warp histograms: the leading digits of nearby scores are all
-            // equal, so one shared counter would serialise every warp.
+        // Range of the keys across the cluster: their common leading bits
+        // (sign, most of the exponent) need no radix pass.
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        }
+        if (lane == 0) {
+            wsum[wid][0] = kmin;
+            wsum[wid][1] = kmax;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t a = 0xffffffffu, z = 0u;
+            for (int i = 0; i < 32; ++i) {
+                a = min(a, wsum[i][0]);
+                z = max(z, wsum[i][1]);
+            }
+            s_cnt[0] = a;
+            s_cnt[1] = z;
+        }
+        csync();
+        uint32_t gmin = 0xffffffffu, gmax = 0u;
+        for (int r = 0; r < NC; ++r) {
+            const uint32_t *rc = remote(&s_cnt[0], r);
+            gmin = min(gmin, rc[0]);
+            gmax = max(gmax, rc[1]);
+        }
+        int hi = 32 - __clz(gmin ^ gmax);                  // bits [hi-1 .. 0] vary
+        pmask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
+        prefix = gmax & pmask;
+        bool use_cand = false;                              // later passes scan only candidates
+        int n_cand = 0;
+        for (int pass = 0; hi > 0; ++pass) {
+            const int wdt = min(8, hi), shift = hi - wdt, buf = pass & 1;
+            const uint32_t dmask = (1u << wdt) - 1u;
             for (int i = tid; i < 32 * 256; i += SEL_THREADS) whist[i >> 8][i & 255] = 0;
             __syncthreads();
-            for (int it = 0; it < seg; it += 32) {
-                const int e = wid * seg + it + lane;
-                const bool valid = e < cnt;
-                const uint32_t key = valid ? key_at(e) : 0u;
-                const bool match = valid && (key & pmask) == prefix;
-                const uint32_t dig = (key >> shift) & 255u;
-                // Usually every matching lane has the same digit: one add by
-                // lane 0; otherwise shared-memory atomics on this warp's copy.
-                const uint32_t mb = __ballot_sync(0xffffffffu, match);
-                const uint32_t d0 = __shfl_sync(0xffffffffu, dig, mb ? __ffs(mb) - 1 : 0);
-                if (__all_sync(0xffffffffu, !match || dig == d0)) {
-                    if (lane == 0 && mb) whist[wid][d0] += (uint32_t)__popc(mb);
-                } else if (match) {
-                    atomicAdd(&whist[wid][dig], 1u);
+            if (use_cand) {
+                for (int ci = tid; ci < n_cand; ci += SEL_THREADS) {
+                    const uint32_t key = cand_key[ci];
+                    if ((key & pmask) == prefix) atomicAdd(&whist[wid][(key >> shift) & dmask], 1u);
                 }
-                __syncwarp();
+            } else {
+                for (int it = 0; it < seg; it += 32) {
+                    const int e = wid * seg + it + lane;
+                    if (e < cnt) {
+                        const uint32_t key = key_at(e);
+                        if ((key & pmask) == prefix) atomicAdd(&whist[wid][(key >> shift) & dmask], 1u);
+                    }
+                }
             }
             __syncthreads();
             if (tid < 256) {
@@ -164,8 +207,32 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
             }
             __syncthreads();
             prefix |= s_digit << shift;
-            pmask |= 255u << shift;
+            pmask |= dmask << shift;
             krem -= s_above;
+            hi = shift;
+            if (pass == 0 && hi > 0) {
+                // Keep the keys that still match: usually a few hundred.
+                if (tid == 0) s_cnt[0] = 0;
+                __syncthreads();
+                for (int it = 0; it < seg; it += 32) {
+                    const int e = wid * seg + it + lane;
+                    const uint32_t key = e < cnt ? key_at(e) : 0u;
+                    const bool m = e < cnt && (key & pmask) == prefix;
+                    const uint32_t mb = __ballot_sync(0xffffffffu, m);
+                    uint32_t base = 0;
+                    if (lane == 0 && mb) base = atomicAdd(&s_cnt[0], (uint32_t)__popc(mb));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const uint32_t pos = base + __popc(mb & ((1u << lane) - 1u));
+                    if (m && pos < (uint32_t)SEL_CAND) {
+                        cand_key[pos] = key;
+                        cand_idx[pos] = (uint32_t)e;
+                    }
+                }
+                __syncthreads();
+                n_cand = (int)s_cnt[0];
+                use_cand = n_cand <= SEL_CAND;
+                __syncthreads();
+            }
         }
     }
     const uint32_t T = prefix;
@@ -270,7 +337,7 @@ cudaError_t launch_select(const CacheView &c, int src, const float *scores, int6
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const int smem = SEL_CAP * (int)sizeof(uint32_t);
+    const int smem = (SEL_CAP + 2 * SEL_CAND) * (int)sizeof(uint32_t);
     if (dev >= 64 || !attr_done[dev]) {
         e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)

@@ -15,10 +15,10 @@ cudaError_t launch_prefill(const CacheView &c, int req, int m, int tok_begin, in
 cudaError_t launch_append(const CacheView &c, const float *lat, const float *key, const float *gate,
                           const int32_t *n_new, cudaStream_t st);
 cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                          void *out, int out_is_fp32, float *part_o, float *part_ml, cudaStream_t st);
+                          void *out, int out_is_fp32, uint32_t flags, float *part_o, float *part_ml, cudaStream_t st);
 
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                               void *out, int out_is_fp32, float *part_o, cudaStream_t st);
+                               void *out, int out_is_fp32, uint32_t flags, float *part_o, cudaStream_t st);
 
 constexpr int ATT_KEYS_PER_SPLIT = 128;
 constexpr int ATT_SPLITS = (CSA2_TOPK + CSA2_SWA) / ATT_KEYS_PER_SPLIT;   // 5: four top-k tiles + the window

@@ -16,7 +16,7 @@ from typing import List, Optional
 import torch
 
 import synth
-from . import (INDEX_FLAT, INDEX_FULL, INDEX_REINDEX, PAGE_CODES_BYTES, PAGE_ENTRIES, PAGE_KEYS_BYTES,
+from . import (ATTEND_INPUTS_SETTLED, INDEX_FLAT, INDEX_FULL, INDEX_REINDEX, PAGE_CODES_BYTES, PAGE_ENTRIES, PAGE_KEYS_BYTES,
                PAGE_SCALES_BYTES, PAGE_SUMM_BYTES, POOL, SWA_CODES_OFF, SWA_SCALE_OFF, TOPK, Cache, csa2_append,
                csa2_attend, csa2_index, csa2_prefill, plane_offsets, workspace)
 
@@ -87,7 +87,10 @@ class DeviceWorkload:
                 grp = 1
                 csa2_index(c, INDEX_REINDEX, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws, stream)
             self.layer_topk.append(grp)
-            csa2_attend(c, q, self.topk[grp], SOFTMAX_SCALE, self.outs[li], self.ws, stream)
+            # A Reuse layer's indices were produced by its group's first layer,
+            # not by the kernel right before it: its gather may start early.
+            flags = ATTEND_INPUTS_SETTLED if mode == "reuse" else 0
+            csa2_attend(c, q, self.topk[grp], SOFTMAX_SCALE, self.outs[li], self.ws, stream, flags=flags)
 
     # ------------------------------------------------------------ read-back
     def entry_rows(self, b: int, entries: torch.Tensor):

@@ -198,10 +198,19 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode,
  * no de-duplication.  q bf16 [batch][heads][512]; heads in 1..128.
  * out [batch][heads][512] is bf16 (out_is_fp32 = 0) or f32 (= 1).  A request
  * with no keys gets a zero output.  Reuse layers call this with their
- * group's topk and their own q. */
+ * group's topk and their own q (and may pass CSA2_ATTEND_INPUTS_SETTLED). */
 csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *q,
                         const int32_t *topk, float scale, void *out, int32_t out_is_fp32,
-                        void *ws, size_t ws_bytes, csa2_stream_t stream);
+                        uint32_t flags, void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* csa2_attend flags.  CSA2_ATTEND_INPUTS_SETTLED: topk, the cache rows it
+ * names and n_tokens were last written by work that finished before the
+ * kernel launched just before this call on `stream` (for example a Reuse
+ * layer, whose indices come from its group's Full layer).  The kernel may
+ * then gather and dequantise those rows while that previous kernel is still
+ * running; only q is read after it completes.  Without the flag every input
+ * is read after the previous kernel completes. */
+#define CSA2_ATTEND_INPUTS_SETTLED 1u
 
 /* Attention without a workspace ------------------------------------------
  * The pages have no counterpart to this call; it exists for callers that

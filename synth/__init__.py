@@ -218,3 +218,24 @@ def page_table(w: Workload) -> torch.Tensor:
         pt[b, : per[b]] = order[off: off + per[b]].to(torch.int32)
         off += per[b]
     return pt
+
+
+def token_rows(w: Workload, b: int, positions, device="cpu", chan: Optional[torch.Tensor] = None):
+    """Raw tokens at arbitrary positions of request b (each chunk drawn once):
+    (lat [n,512], key [n,128], gate [n]) in the order given."""
+    pos = torch.as_tensor(positions, dtype=torch.int64).reshape(-1)
+    if chan is None:
+        chan = channel_scale(w)
+    chan = chan.to(device)
+    lat = torch.empty(pos.numel(), LATENT, device=device)
+    key = torch.empty(pos.numel(), IDX_DIM, device=device)
+    gate = torch.empty(pos.numel(), device=device)
+    chunks = pos // CHUNK
+    for c in torch.unique(chunks).tolist():
+        sel = torch.nonzero(chunks == c).reshape(-1)
+        l_, k_, g_ = tokens(w, b, c * CHUNK, c * CHUNK + CHUNK, device, chan)
+        off = (pos[sel] - c * CHUNK).to(device)
+        lat[sel.to(device)] = l_[off]
+        key[sel.to(device)] = k_[off]
+        gate[sel.to(device)] = g_[off]
+    return lat, key, gate

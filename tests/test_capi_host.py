@@ -62,21 +62,22 @@ def test_invalid_arguments_rejected_before_launch(csa2):
     # cache with a null field / zero batch
     for kw in ({"pool": None}, {"batch": 0}, {"n_pages": 0}, {"max_pages": 0}, {"pool": 256 * 1000 + 8}):
         c = _fake_cache(csa2, **kw)
-        assert L.csa2_attend(C.byref(c), 64, good, good, 0.1, good, 0, good, 1 << 30, None) == 1, kw
+        assert L.csa2_attend(C.byref(c), 64, good, good, 0.1, good, 0, 0, good, 1 << 30, None) == 1, kw
     c = _fake_cache(csa2)
     # bad mode, bad heads, missing pool in FULL mode, workspace too small
     assert L.csa2_index(C.byref(c), 7, good, good, good, good, good, good, 1 << 30, None) == 1
-    assert L.csa2_attend(C.byref(c), 0, good, good, 0.1, good, 0, good, 1 << 30, None) == 1
-    assert L.csa2_attend(C.byref(c), 129, good, good, 0.1, good, 0, good, 1 << 30, None) == 1
+    assert L.csa2_attend(C.byref(c), 0, good, good, 0.1, good, 0, 0, good, 1 << 30, None) == 1
+    assert L.csa2_attend(C.byref(c), 129, good, good, 0.1, good, 0, 0, good, 1 << 30, None) == 1
     assert L.csa2_index(C.byref(c), 1, good, good, None, None, good, good, 1 << 30, None) == 1
     assert L.csa2_index(C.byref(c), 0, good, good, None, None, good, good, 16, None) == 1
-    assert L.csa2_attend(C.byref(c), 64, good, good, 0.1, good, 0, good, 16, None) == 1
+    assert L.csa2_attend(C.byref(c), 64, good, good, 0.1, good, 0, 0, good, 16, None) == 1
     # prefill: bad request, m, alignment, range, capacity
     assert L.csa2_prefill(C.byref(c), 5, 1, 0, 10, 10, good, good, good, None) == 1
     assert L.csa2_prefill(C.byref(c), 0, 3, 0, 10, 10, good, good, good, None) == 1
     assert L.csa2_prefill(C.byref(c), 0, 2, 1, 10, 20, good, good, good, None) == 1
     assert L.csa2_prefill(C.byref(c), 0, 1, 0, 10, 5, good, good, good, None) == 1
     assert L.csa2_prefill(C.byref(c), 0, 1, 0, 300, 300, good, good, good, None) == 1   # 4 pages = 256 entries
+    assert L.csa2_attend(C.byref(c), 64, good, good, 0.1, good, 0, 6, good, 1 << 30, None) == 1   # unknown flag
     assert L.csa2_append(C.byref(c), None, good, good, good, None) == 1
     assert L.csa2_get_device_error(None, None, None) == 1
     assert csa2.status_string(1) == "invalid argument"
