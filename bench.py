@@ -42,6 +42,21 @@ FLUSH_BYTES = 256 << 20
 
 
 # ------------------------------------------------------------------ helpers
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest `value` across ranks (the slowest rank's device time)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, batch_per_rank: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job queries/s: every rank decodes its own batch each step
+    (replicas, weak scaling); the slowest rank's time counts."""
+    return world * batch_per_rank * steps / (max_total_ms / 1e3)
+
+
 def algorithmic_bytes(w: synth.Workload) -> dict:
     """Bytes the step must move, per the layout (per request, summed):
     index  FULL: ceil(N/8)*128 [if > 2048 blocks] + min(N,16384)*128 + 16384*4
@@ -319,13 +334,8 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_total_ms = float(t.item())
-    queries = world * w.batch * args.steps
-    value = queries / (max_total_ms / 1e3)
+    max_total_ms = max_over_ranks(sum(step_ms), world, dev)
+    value = job_throughput(world, w.batch, args.steps, max_total_ms)
 
     # ---- end to end: pinned host inputs -> device, replay, outputs -> host
     ins = [x for li, mode in enumerate(w.layers) for x in
@@ -354,10 +364,7 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
         stream.synchronize()
         if i >= 3:
             e2e_ms.append(a.elapsed_time(b))
-    te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = world * w.batch * e2e_steps / (float(te.item()) / 1e3)
+    e2e_value = job_throughput(world, w.batch, e2e_steps, max_over_ranks(sum(e2e_ms), world, dev))
 
     # ---- roofline of the dominant kernel (live CUDA-event timing)
     ab = algorithmic_bytes(w)
@@ -380,7 +387,7 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
         cpu = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
         line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": step_avg_ms, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+                "vs_baseline": None, "dtype": "fp8/bf16 MMA, fp32 accumulate", "data": "synthetic",
                 "config": {"workload": w.name, "batch_per_gpu": w.batch, "entries_per_request": w.n_entries[0],
                            "heads": w.heads, "layers": w.layers, "index": w.index,
                            "l2": "flushed between timed steps (256 MB write, not timed)",
