@@ -86,6 +86,29 @@ def algorithmic_bytes(w: synth.Workload) -> dict:
     return tot
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# the ncu captures summarised under profiles/, valid only while the kernel's
+# source is the one that was captured.
+KNOWN_TRAFFIC = {
+    "block_scan": {"bytes": 67_516_672 + 708_352, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
+                   "sha256": "b77b9fe65da6cd45aa0ca2cee1e9157ad4314ea23007d4f8f3957fe5666615a4"},
+}
+
+
+def known_traffic(name: str):
+    t = KNOWN_TRAFFIC.get(name)
+    if t is None:
+        return None
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, t["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != t["sha256"]:
+                return None
+    except OSError:
+        return None
+    return t["bytes"]
+
+
 def measured_peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -146,6 +169,14 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bench_config(w: synth.Workload) -> dict:
+    """The workload description both arms print."""
+    return {"workload": w.name, "batch_per_gpu": w.batch, "entries_per_request": w.n_entries[0],
+            "heads": w.heads, "layers": w.layers, "index": w.index,
+            "l2": "flushed between timed steps (256 MB write, not timed)",
+            "timing": "CUDA graph replay of one step, CUDA events per step"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) side
@@ -259,8 +290,7 @@ def run_reference(args, w: synth.Workload, rank: int, world: int):
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": 1, "sample": "one request, stage units round-robin"},
-            "impl": "reference",
+            "config": bench_config(w), "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
                              "sample": f"each step = one of the {U} stage units of one request's decode step "
                                        f"(round-robin; {U} steps = one query)"},
@@ -278,9 +308,9 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
     dw = DeviceWorkload(w, dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
-    dom_kernel = csa2.KERNEL_FLAT_SCORE if w.index == "flat" else csa2.KERNEL_BLOCK_SCORE
-    k_start = torch.cuda.Event(enable_timing=True)
-    k_stop = torch.cuda.Event(enable_timing=True)
+    k_scan = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    k_att = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    n_layers = len(w.layers)
 
     # warm up eagerly once (first-call attribute set-up happens outside capture)
     with torch.cuda.stream(stream):
@@ -290,31 +320,38 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
     assert csa2.csa2_get_device_error(dw.cache, stream) == 0
 
     # torch only reports elapsed time between events it has recorded itself;
-    # record the pair once so later records by the library are readable.
-    k_start.record(stream)
-    k_stop.record(stream)
+    # record each pair once so later records by the library are readable.
+    for ev in k_scan + k_att:
+        ev.record(stream)
     stream.synchronize()
-    csa2.csa2_set_profile_events(dom_kernel, k_start, k_stop)
-    graph = torch.cuda.CUDAGraph()
+    # One graph per layer: graph L brackets the attention of layer L (and the
+    # index scan) with events, so the timed replays, taken in turn, measure
+    # every layer's attention launch equally often.
+    scan_kernel = csa2.KERNEL_FLAT_SCORE if w.index == "flat" else csa2.KERNEL_BLOCK_SCORE
+    csa2.csa2_set_profile_events(scan_kernel, *k_scan)
+    graphs = []
     n0 = csa2.csa2_launch_count()
-    with torch.cuda.graph(graph, stream=stream):
-        dw.step(stream)
-    launches_per_step = csa2.csa2_launch_count() - n0
-    csa2.csa2_set_profile_events(dom_kernel, None, None)
+    for li in range(n_layers):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            dw.step(stream, attend_events=(li, k_att[0], k_att[1]))
+        graphs.append(g)
+    launches_per_step = (csa2.csa2_launch_count() - n0) / n_layers
+    csa2.csa2_set_profile_events(scan_kernel, None, None)
 
-    def one(timed_events=None):
+    def one(i, timed_events=None):
         with torch.cuda.stream(stream):
             if w.append:
                 dw.restore(stream)
             flush.zero_()
             if timed_events:
                 timed_events[0].record(stream)
-            graph.replay()
+            graphs[i % n_layers].replay()
             if timed_events:
                 timed_events[1].record(stream)
 
-    for _ in range(max(args.warmup, 3)):
-        one()
+    for i in range(max(args.warmup, 3)):
+        one(i)
     stream.synchronize()
 
     sampler = ClockSampler(local_rank)
@@ -322,14 +359,15 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
-    step_ms, kern_ms = [], []
+    step_ms, scan_ms, att_ms = [], [], []
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
     for i in range(args.steps):
         e = ev[i % 2]
-        one(e)
+        one(i, e)
         stream.synchronize()
         step_ms.append(e[0].elapsed_time(e[1]))
-        kern_ms.append(k_start.elapsed_time(k_stop))
+        scan_ms.append(k_scan[0].elapsed_time(k_scan[1]))
+        att_ms.append(k_att[0].elapsed_time(k_att[1]))
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -357,7 +395,7 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
             a.record(stream)
             for d, h in zip(ins, host_in):
                 d.copy_(h, non_blocking=True)
-            graph.replay()
+            graphs[i % n_layers].replay()
             for h, o in zip(host_out, dw.outs):
                 h.copy_(o, non_blocking=True)
             b.record(stream)
@@ -366,21 +404,32 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
             e2e_ms.append(a.elapsed_time(b))
     e2e_value = job_throughput(world, w.batch, e2e_steps, max_over_ranks(sum(e2e_ms), world, dev))
 
-    # ---- roofline of the dominant kernel (live CUDA-event timing)
+    # ---- roofline: attention (the largest share of the step's kernel time)
+    # and the index scan, both timed live with CUDA events on the launching
+    # stream over the timed region
     ab = algorithmic_bytes(w)
-    kbytes = ab["block_summaries"] if w.index != "flat" else ab["index"]
-    kern_avg_ms = statistics.mean(kern_ms)
-    achieved = kbytes / (kern_avg_ms / 1e3) / 1e9
     peak, peak_src = measured_peak_hbm()
     step_avg_ms = max_total_ms / args.steps
-    roofline = {"bound": "hbm", "kernel": "block_score" if w.index != "flat" else "flat_score",
-                "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None,
-                "kernel_ms": kern_avg_ms, "kernel_share_of_step": kern_avg_ms / step_avg_ms,
-                "algorithmic_bytes_per_launch": kbytes,
+    att_avg_ms = statistics.mean(att_ms)
+    att_bytes = ab["attend"] / n_layers
+    att_gbs = att_bytes / (att_avg_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "attend_dsm_kernel", "achieved": att_gbs, "peak": peak,
+                "peak_source": peak_src, "unit": "GB/s", "frac": att_gbs / peak,
+                "traffic": known_traffic("attend"),
+                "kernel_ms": att_avg_ms, "launches_per_step": n_layers,
+                "kernel_share_of_step": att_avg_ms * n_layers / step_avg_ms,
+                "algorithmic_bytes_per_launch": att_bytes,
                 "step_achieved_gbs": ab["step"] / (step_avg_ms / 1e3) / 1e9,
                 "step_frac": ab["step"] / (step_avg_ms / 1e3) / 1e9 / peak,
                 "step_algorithmic_bytes": ab["step"]}
+    scan_avg_ms = statistics.mean(scan_ms)
+    scan_bytes = ab["block_summaries"] if w.index != "flat" else ab["index"]
+    scan_gbs = scan_bytes / (scan_avg_ms / 1e3) / 1e9
+    roofline_scan = {"bound": "hbm", "kernel": "score_umma_kernel (block-summary scan)" if w.index != "flat"
+                     else "score_umma_kernel (flat key scan)", "achieved": scan_gbs, "peak": peak,
+                     "peak_source": peak_src, "unit": "GB/s", "frac": scan_gbs / peak,
+                     "traffic": known_traffic("block_scan") if w.index != "flat" else None,
+                     "kernel_ms": scan_avg_ms, "algorithmic_bytes_per_launch": scan_bytes}
 
     line = None
     if rank == 0:
@@ -388,17 +437,14 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
         line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": step_avg_ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "fp8/bf16 MMA, fp32 accumulate", "data": "synthetic",
-                "config": {"workload": w.name, "batch_per_gpu": w.batch, "entries_per_request": w.n_entries[0],
-                           "heads": w.heads, "layers": w.layers, "index": w.index,
-                           "l2": "flushed between timed steps (256 MB write, not timed)",
-                           "timing": "CUDA graph replay of one step, CUDA events per step"},
-                "roofline": roofline, "cpu_baseline": cpu,
+                "config": bench_config(w),
+                "roofline": roofline, "roofline_index_scan": roofline_scan, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": int(launches_per_step * args.steps),
                 "clocks": clocks}
         print(json.dumps(line), flush=True)
-    del graph
+    del graphs
     return line
 
 

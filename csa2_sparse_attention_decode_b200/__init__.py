@@ -31,7 +31,7 @@ INDEX_FLAT, INDEX_FULL, INDEX_REINDEX = 0, 1, 2
 
 EXPORTS = ("csa2_page_bytes", "csa2_swa_bytes", "csa2_workspace_bytes", "csa2_prefill", "csa2_append",
            "csa2_index", "csa2_attend", "csa2_get_device_error", "csa2_status_string", "csa2_set_profile_events",
-           "csa2_launch_count", "csa2_attend_noalloc")
+           "csa2_launch_count", "csa2_attend_noalloc", "csa2_topk")
 ATTEND_NOALLOC_MAX_ROWS = 512
 KERNEL_BLOCK_SCORE, KERNEL_FLAT_SCORE, KERNEL_POOL_SCORE, KERNEL_SELECT, KERNEL_ATTEND, KERNEL_COMBINE = range(6)
 
@@ -71,6 +71,7 @@ def _load():
         "csa2_set_profile_events": (C.c_int, [I32, P, P]),
         "csa2_attend_noalloc": (C.c_int, [P, I32, P, P, C.c_float, P, I32, P]),
         "csa2_launch_count": (C.c_uint64, []),
+        "csa2_topk": (C.c_int, [P, C.c_int64, P, I32, I32, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -174,6 +175,15 @@ def csa2_index(cache: Cache, mode: int, q_idx, w, pool, pool_len, topk, ws, stre
     qi = q_idx.view(torch.int16) if q_idx.dtype == torch.bfloat16 else q_idx
     _check("csa2_index", lib.csa2_index(cache.ref, mode, _ptr(qi), _ptr(w), _ptr(pool), _ptr(pool_len),
                                         _ptr(topk), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def csa2_topk(scores, n, k: int, out, stream=None):
+    """Top-k of each row of scores [batch, stride] (f32), first n[b] elements
+    (n int32 [batch]); out int32 [batch, k] gets ascending indices, -1 padded."""
+    assert scores.dtype == torch.float32 and scores.stride(1) == 1 and n.dtype == torch.int32
+    assert out.dtype == torch.int32 and out.is_contiguous() and tuple(out.shape) == (scores.shape[0], k)
+    _check("csa2_topk", lib.csa2_topk(_ptr(scores), scores.stride(0), _ptr(n), int(scores.shape[0]), int(k),
+                                      _ptr(out), _stream(stream)))
 
 
 ATTEND_INPUTS_SETTLED = 1

@@ -8,7 +8,8 @@
 // once it is running (an allocation can synchronise the device and stall
 // every stream).  This entry point keeps the partials in a fixed array that
 // is part of the library itself, so the caller passes only inputs and
-// outputs.  It launches the same kernels as csa2_attend.
+// outputs.  It launches the attention variant that exchanges its split
+// partials through global memory (csa2_attend merges them on chip instead).
 #include <mutex>
 
 #include "common.cuh"
@@ -17,12 +18,11 @@
 namespace {
 
 constexpr size_t kPartO = (size_t)CSA2_ATTEND_NOALLOC_MAX_ROWS * csa2::ATT_SPLITS * CSA2_LATENT;
-constexpr size_t kPartML = (size_t)CSA2_ATTEND_NOALLOC_MAX_ROWS * csa2::ATT_SPLITS * 2;
 
 // One copy per GPU that loads the library, held until the process exits.
 // Host code must not use this name as a pointer: on the host it is only a
 // stand-in, and its device address comes from cudaGetSymbolAddress below.
-static __device__ __align__(256) float g_attend_scratch[kPartO + kPartML];
+static __device__ __align__(256) float g_attend_scratch[kPartO];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
@@ -68,9 +68,7 @@ extern "C" csa2_status csa2_attend_noalloc(const csa2_cache *cache, int32_t head
     if (scratch_address(&scratch) != cudaSuccess) return CSA2_ERR_CUDA;
     // Every partial the combine step reads is written by this same call, so
     // nothing left over from an earlier call needs clearing.
-    float *part_o = scratch;
-    float *part_ml = scratch + kPartO;
-    cudaError_t e = csa2::launch_attend(csa2::make_view(cache), heads, q, topk, scale, out, out_is_fp32, 0u, part_o,
-                                        part_ml, (cudaStream_t)stream);
+    cudaError_t e = csa2::launch_attend_umma(csa2::make_view(cache), heads, q, topk, scale, out, out_is_fp32, 0u,
+                                             scratch, (cudaStream_t)stream);
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

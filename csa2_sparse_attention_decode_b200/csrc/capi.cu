@@ -146,11 +146,20 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
                               W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, max_blocks, s);
         if (e != cudaSuccess) return from_cuda(e);
     }
-    e = launch_score(c, ROWS_POOL, q_idx, w, pool, pool_len, W.scores_b, CSA2_POOL, CSA2_POOL, s);
-    if (e == cudaSuccess)
-        e = launch_select(c, ROWS_POOL, W.scores_b, CSA2_POOL, pool_len, pool, CSA2_TOPK, topk, CSA2_TOPK, 0,
-                          nullptr, nullptr, CSA2_POOL, s);
-    return from_cuda(e);
+    return from_cuda(launch_pool_select(c, q_idx, w, pool, pool_len, topk, s));
+}
+
+csa2_status csa2_topk(const float *scores, int64_t stride, const int32_t *n, int32_t batch, int32_t k,
+                      int32_t *out, csa2_stream_t stream)
+{
+    if (!scores || !n || !out || batch <= 0 || batch > 65535 || k < 1 || k > CSA2_MAX_BLOCKS || stride < 1)
+        return CSA2_ERR_INVALID_ARG;
+    if (stride > ((int64_t)1 << 31) / batch) return CSA2_ERR_INVALID_ARG;
+    CacheView c = {};
+    c.batch = batch;
+    const int max_n = stride > (int64_t)(1 << 30) ? (1 << 30) : (int)stride;
+    return from_cuda(launch_select(c, ROWS_GIVEN, scores, stride, n, nullptr, k, out, k, 0, nullptr, nullptr, max_n,
+                                   (cudaStream_t)stream));
 }
 
 csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *q, const int32_t *topk, float scale,

@@ -3,13 +3,17 @@
 #include "common.cuh"
 
 namespace csa2 {
-enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2 };
+enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2, ROWS_GIVEN = 3 };
 
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,
                          const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st);
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
                           int32_t *pool_len, int max_n, cudaStream_t st);
+// Exact rescoring of the pool fused with its top-512 selection (one cluster
+// per request); writes the selected pool ids, ascending, -1 padded.
+cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const float *w, const int32_t *pool,
+                               const int32_t *pool_len, int32_t *topk, cudaStream_t st);
 cudaError_t launch_prefill(const CacheView &c, int req, int m, int tok_begin, int n_tok, int n_tok_final,
                            const float *lat, const float *key, const float *gate, cudaStream_t st);
 cudaError_t launch_append(const CacheView &c, const float *lat, const float *key, const float *gate,
@@ -17,6 +21,12 @@ cudaError_t launch_append(const CacheView &c, const float *lat, const float *key
 cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
                           void *out, int out_is_fp32, uint32_t flags, float *part_o, float *part_ml, cudaStream_t st);
 
+// Attention with the split merge inside a cluster (distributed shared memory):
+// the csa2_attend path.  Needs no scratch.
+cudaError_t launch_attend_dsm(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
+                              void *out, int out_is_fp32, uint32_t flags, cudaStream_t st);
+// Attention with the scaled split partials exchanged through global scratch
+// `part_o` ([batch][5][heads][512] fp32): the csa2_attend_noalloc path.
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
                                void *out, int out_is_fp32, uint32_t flags, float *part_o, cudaStream_t st);
 

@@ -8,16 +8,14 @@
 //   warp 4      TMA producer: 128-row tiles (16 KB of FP8) into a 5-stage
 //               shared-memory ring, 128-byte swizzled, one box per page run.
 //   warp 5      allocates tensor memory and issues the MMAs straight on the
-//               FP8 tile: D[128 x 96] (fp32) = K[128 x 128] (e4m3) . Qs^T,
-//               kind::f8f6f4, where Qs stacks three e5m2 parts of the query
-//               (32 heads each); their sum is the query exactly (see below).
+//               FP8 tile: D[128 x 32] (fp32) = sum_p K[128 x 128] (e4m3) .
+//               Qp^T, kind::f8f6f4, where Q1 + Q2 + Q3 is the query split
+//               exactly into three e5m2 parts (idx_query.cuh); the tensor
+//               cores add the three products into one accumulator.  Four
+//               accumulators of 32 columns let the MMAs run ahead of the
+//               epilogue.
 //   warps 0-3   convert the query once per request; thread = row epilogue:
-//               dot_h = D[h] + D[32+h] + D[64+h], score = sum_h w'_h ReLU(dot_h).
-// Query split: per head, q' = q * 2^s with max|q'| in [2^14, 2^15); then
-// q' = p1 + p2 + p3 with p1 = e5m2(q'), p2 = e5m2(q' - p1), p3 = e5m2(rest).
-// A bf16 value has 8 significant bits and each e5m2 part takes 3, so the sum
-// is exact for every element not below 2^-9 (e5m2 steps of 2^-16), i.e. down
-// to 2^-24 of the head's largest entry; w'_h = w_h * 2^-s undoes the scale.
+//               score = sum_h w'_h ReLU(D[h]).
 // The tensor cores accumulate these products at fp32 precision (checked on
 // hardware against exact sums), so the scores are fp32-accumulated
 // sum_h w_h ReLU(q_h . k) as the method defines them.
@@ -26,6 +24,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "idx_query.cuh"
 #include "index.cuh"
 #include "umma.cuh"
 
@@ -39,15 +38,16 @@ constexpr int STAGES = 5;
 constexpr int CTAS_PER_SM = 2;                              // two independent pipelines per SM
 constexpr int PW = 16;                                      // producer look-up window (tiles)
 constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;            // 16 KB
-constexpr int QPARTS = 3;
-constexpr int QROWS = QPARTS * CSA2_IDX_HEADS;              // 96 = MMA N
-constexpr int QBYTES = QROWS * CSA2_KEY_DIM;                // 12 KB of e5m2
+constexpr int QBYTES = IQ_BYTES;                            // 3 parts x 32 heads x 128 dims of e5m2
+constexpr int QPART_BYTES = CSA2_IDX_HEADS * CSA2_KEY_DIM;  // 4 KB: one part
+constexpr int ACC = 4;                                      // accumulators in tensor memory
+constexpr int ACC_COLS = CSA2_IDX_HEADS;                    // 32 columns each
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;                         // D: 2 x 96 columns
+constexpr uint32_t TMEM_COLS = ACC * ACC_COLS;              // 128
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + QBYTES;   // + 8 * (batch + 1)
 constexpr int MAX_BATCH = 1024;
-// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, N = 96, M = 128.
-constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(QROWS >> 3) << 17) | (8u << 24);
+// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, N = 32, M = 128.
+constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(ACC_COLS >> 3) << 17) | (8u << 24);
 
 // 2-D views (rows of 128 bytes) of the summary and key planes, with boxes of
 // one 8-row run, one 64-row page and one whole 128-row tile.
@@ -132,11 +132,6 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
                  : "memory");
 }
 
-__device__ __forceinline__ float e5m2_to_f32(uint8_t c)
-{
-    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E5M2);
-    return __half2float(__half(h));
-}
 
 __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
 score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
@@ -144,7 +139,7 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *qbuf = sm + STAGES * STAGE_BYTES;
-    __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], d_full[2], d_empty[2], q_full;
+    __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], d_full[ACC], d_empty[ACC], q_full;
     __shared__ float wq[CSA2_IDX_HEADS];
     __shared__ uint32_t tmem_base;
     __shared__ long long s_total;
@@ -158,7 +153,7 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < ACC; ++i) {
             mbar_init(&d_full[i], 1);
             mbar_init(&d_empty[i], 4);
         }
@@ -335,12 +330,12 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         int cur_b = -1, sw = -1, issued = 0;
         const uint32_t qaddr = smem_addr(qbuf);
         for (int j = 0; j < n_items; ++j, it.next()) {
-            const int ab = j & 1, s = j % STAGES;
+            const int ab = j % ACC, s = j % STAGES;
             bool okw = true;
             if (lane == 0) {
                 if (it.b != cur_b) okw = wait_or_abort(&q_full, (sw + 1) & 1, abort, p.c.error);
                 if (okw) okw = wait_or_abort(&full[s], (j / STAGES) & 1, abort, p.c.error);
-                if (okw && j >= 2) okw = wait_or_abort(&d_empty[ab], ((j >> 1) - 1) & 1, abort, p.c.error);
+                if (okw && j >= ACC) okw = wait_or_abort(&d_empty[ab], ((j / ACC) - 1) & 1, abort, p.c.error);
             }
             if (it.b != cur_b) {
                 cur_b = it.b;
@@ -352,8 +347,10 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
                 const uint32_t aaddr = smem_addr(sm + s * STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < CSA2_KEY_DIM / 32; ++kk)
-                    mma_f8(tb + QROWS * ab, smem_desc(aaddr + kk * 32, 16, 1024), smem_desc(qaddr + kk * 32, 16, 1024),
-                           IDESC, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int pp = 0; pp < IQ_PARTS; ++pp)
+                        mma_f8(tb + ACC_COLS * ab, smem_desc(aaddr + kk * 32, 16, 1024),
+                               smem_desc(qaddr + pp * QPART_BYTES + kk * 32, 16, 1024), IDESC, (kk | pp) ? 1u : 0u);
                 mma_commit(&d_full[ab]);
                 mma_commit(&empty[s]);                              // stage free once the MMAs have read it
             }
@@ -361,7 +358,7 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             issued = j + 1;
         }
         if (lane == 0)
-            for (int j = max(0, issued - 2); j < issued; ++j) mbar_wait(&d_full[j & 1], (j >> 1) & 1);
+            for (int j = max(0, issued - ACC); j < issued; ++j) mbar_wait(&d_full[j % ACC], (j / ACC) & 1);
         __syncwarp();
     } else if (warp < 4 && n_items > 0) {
         // ------------------------------------------------------------ workers
@@ -369,86 +366,33 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         it.init(s_rows, s_pre, p.c.batch, i0, i1);
         const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
         int cur_b = -1;
+        float wr[CSA2_IDX_HEADS];                                  // this request's w'
         for (int j = 0; j < n_items; ++j, it.next()) {
             if (it.b != cur_b) {
                 // New request.  Every MMA issued so far has completed (the
                 // previous epilogue waited for it), so the q buffer is free.
                 cur_b = it.b;
-                const int h = tid >> 2, qd = tid & 3;
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.q_idx + ((size_t)cur_b * CSA2_IDX_HEADS + h) *
-                                                                                 CSA2_KEY_DIM + 32 * qd);
-                uint4 raw[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) raw[i] = src[i];
-                const uint32_t *rw = reinterpret_cast<const uint32_t *>(raw);
-                float x[32];
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    x[2 * i] = __uint_as_float(rw[i] << 16);
-                    x[2 * i + 1] = __uint_as_float(rw[i] & 0xffff0000u);
-                    amax = fmaxf(amax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
-                }
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                int ex = 0;
-                if (amax > 0.0f) frexpf(amax, &ex);
-                const int sh = (amax > 0.0f) ? 15 - ex : 0;          // amax * 2^sh in [2^14, 2^15)
-                uint32_t part[QPARTS][8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    uint32_t w0 = 0, w1 = 0, w2 = 0;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float r = ldexpf(x[4 * i + k], sh);
-                        const uint8_t c0 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
-                        r -= e5m2_to_f32(c0);
-                        const uint8_t c1 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
-                        r -= e5m2_to_f32(c1);
-                        const uint8_t c2 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
-                        w0 |= (uint32_t)c0 << (8 * k);
-                        w1 |= (uint32_t)c1 << (8 * k);
-                        w2 |= (uint32_t)c2 << (8 * k);
-                    }
-                    part[0][i] = w0;
-                    part[1][i] = w1;
-                    part[2][i] = w2;
-                }
-                // row n = part * 32 + h, bytes 32*qd .. +31 = 16-byte chunks 2qd, 2qd+1
-#pragma unroll
-                for (int pp = 0; pp < QPARTS; ++pp) {
-                    const int n = pp * CSA2_IDX_HEADS + h;
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        const int chunk = 2 * qd + cc;
-                        *reinterpret_cast<uint4 *>(qbuf + n * 128 + ((chunk ^ (n & 7)) << 4)) =
-                            make_uint4(part[pp][4 * cc], part[pp][4 * cc + 1], part[pp][4 * cc + 2],
-                                       part[pp][4 * cc + 3]);
-                    }
-                }
-                if (qd == 0) wq[h] = ldexpf(p.w[(size_t)cur_b * CSA2_IDX_HEADS + h], -sh);
+                iq_split(tid, p.q_idx, p.w, cur_b, qbuf, wq);
                 fence_proxy_async_smem();
                 bar_workers();
                 if (tid == 0) mbar_arrive(&q_full);
+#pragma unroll
+                for (int hh = 0; hh < CSA2_IDX_HEADS; ++hh) wr[hh] = wq[hh];
             }
             // ---- epilogue of tile j
-            const int db = j & 1;
-            const bool ok = wait_or_abort(&d_full[db], (j >> 1) & 1, abort, p.c.error);
+            const int db = j % ACC;
+            const bool ok = wait_or_abort(&d_full[db], (j / ACC) & 1, abort, p.c.error);
             fence_after_sync();
-            uint32_t r0[32], r1[32], r2[32];
-            tmem_ld32(tb + lane_base + QROWS * db, r0);
-            tmem_ld32(tb + lane_base + QROWS * db + 32, r1);
-            tmem_ld32(tb + lane_base + QROWS * db + 64, r2);
+            uint32_t r0[32];
+            tmem_ld32(tb + lane_base + ACC_COLS * db, r0);
             tmem_ld_wait();
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&d_empty[db]);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int hh = 0; hh < CSA2_IDX_HEADS; ++hh) {
-                const float dot = (__uint_as_float(r0[hh]) + __uint_as_float(r1[hh])) + __uint_as_float(r2[hh]);
-                acc[hh & 3] = fmaf(wq[hh], fmaxf(dot, 0.0f), acc[hh & 3]);
-            }
+            for (int hh = 0; hh < CSA2_IDX_HEADS; ++hh)
+                acc[hh & 3] = fmaf(wr[hh], fmaxf(__uint_as_float(r0[hh]), 0.0f), acc[hh & 3]);
             const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             const int row = it.t * TILE + tid;
             if (ok && row < it.rows) p.scores[(size_t)it.b * p.stride + row] = sc;

@@ -1,0 +1,353 @@
+// Exact top-k selection over order-preserving 32-bit keys held in shared
+// memory, for one CTA or one thread-block cluster of NC CTAs (each CTA owns a
+// contiguous range of the elements).  Score descending, ties to the lower
+// index, output in ascending index order.
+//
+// Method (a radix select):
+//   1. the cluster-wide min and max key give the leading bits every key
+//      shares; no pass is spent on them;
+//   2. one 8-bit histogram pass over the next bits finds the bin that holds
+//      the k-th largest key and how many keys of that bin to take (krem);
+//   3. the keys of that bin (the candidates, usually a few hundred) are
+//      compacted.  When the cluster holds at most RANK_MAX of them, each
+//      candidate is ranked directly against all candidates (key desc, index
+//      asc) and marked when its rank is below krem.  Otherwise further 8-bit
+//      passes over the candidates (or all keys, if they overflowed) find the
+//      exact threshold key T, and the first krem keys equal to T in index
+//      order are taken;
+//   4. a counting pass and an ordered compaction write the selected ids.
+// Histograms, counts and candidates are exchanged over distributed shared
+// memory.  Used by the top-k kernels of index.cu and by the fused pool
+// rescoring kernel.
+#pragma once
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace csa2 {
+namespace sel {
+
+namespace cg = cooperative_groups;
+
+constexpr int CAND = 2048;       // candidates a CTA keeps after the first pass
+constexpr int RANK_MAX = 2048;   // cluster-wide candidates ranked directly
+
+// Order-preserving 32-bit key of an fp32 score (-0 folded onto +0).
+__device__ __forceinline__ uint32_t ord_key(float x)
+{
+    uint32_t u = __float_as_uint(x);
+    if (u == 0x80000000u) u = 0;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Shared-memory work areas the caller provides (dynamic shared memory).
+struct Bufs {
+    const uint32_t *keys;        // [cnt] keys of this CTA's range, or nullptr: read `scores`
+    const float *scores;         // global scores of this CTA's range (when keys == nullptr)
+    uint32_t *cand_key, *cand_idx;    // [CAND]
+    uint32_t *all_key, *all_idx;      // [RANK_MAX]
+    uint32_t *bits;              // [bits_words] selection marks of candidates (local index)
+    int bits_words;
+};
+
+// Where the selected ids go.
+struct Out {
+    int32_t *out;                // out[b*out_stride + pos] (plain / id-mapped mode)
+    int out_stride;
+    const int32_t *ids;          // optional map: the id of element i is ids[b*CSA2_POOL + i]
+    int expand;                  // ids are block numbers: write their entries to pool
+    int32_t *pool, *pool_len;
+    int n_entries;               // entries of the request (expand mode)
+};
+
+// Inclusive scan over threads 0..255 (warps 0..7); every thread of the CTA
+// must call it.  Returns the prefix for threads < 256.
+__device__ __forceinline__ uint32_t scan256(uint32_t v, uint32_t *scratch)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    if (wid < 8 && lane == 31) scratch[wid] = v;
+    __syncthreads();
+    uint32_t add = 0;
+    if (wid < 8)
+        for (int i = 0; i < wid; ++i) add += scratch[i];
+    __syncthreads();
+    return v + add;
+}
+
+// Selects the top min(k, n) of the n elements of request b; CTA r of the NC
+// holds elements [r*chunk, r*chunk + chunk) of them, this one [lo, lo + cnt)
+// with lo = rank*chunk.  kmin / kmax: this thread's
+// min / max over the keys it staged (any split of the range over the
+// threads).  NT = threads per CTA (a multiple of 32, at least 256).
+template <int NC, int NT>
+__device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int chunk, int lo, int cnt, int k,
+                                            uint32_t kmin, uint32_t kmax, const Out &o)
+{
+    constexpr int NW = NT / 32;
+    __shared__ uint32_t hist[2][256];
+    __shared__ uint32_t whist[NW][256];
+    __shared__ uint32_t scratch[32];
+    __shared__ uint32_t wsum[NW][2];
+    __shared__ uint32_t s_cnt[4];
+    __shared__ uint32_t s_digit, s_above;
+    const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
+    auto csync = [&]() {
+        if constexpr (NC > 1) cg::this_cluster().sync();
+        else __syncthreads();
+    };
+    auto remote = [&](uint32_t *ptr, int r) -> uint32_t * {
+        if constexpr (NC > 1) return cg::this_cluster().map_shared_rank(ptr, r);
+        else return ptr;
+    };
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int kk = min(k, n);
+    const bool take_all = n <= k;
+    const int seg = ((cnt + NW * 32 - 1) / (NW * 32)) * 32;     // elements per warp, multiple of 32
+    auto key_at = [&](int e) -> uint32_t { return bf.keys ? bf.keys[e] : ord_key(bf.scores[e]); };
+
+    uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kk;
+    bool ranked = false;                                    // candidates were ranked directly
+    if (!take_all) {
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+        }
+        if (lane == 0) {
+            wsum[wid][0] = kmin;
+            wsum[wid][1] = kmax;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t a = 0xffffffffu, z = 0u;
+            for (int i = 0; i < NW; ++i) {
+                a = min(a, wsum[i][0]);
+                z = max(z, wsum[i][1]);
+            }
+            s_cnt[0] = a;
+            s_cnt[1] = z;
+        }
+        csync();
+        uint32_t gmin = 0xffffffffu, gmax = 0u;
+        for (int r = 0; r < NC; ++r) {
+            const uint32_t *rc = remote(&s_cnt[0], r);
+            gmin = min(gmin, rc[0]);
+            gmax = max(gmax, rc[1]);
+        }
+        int hi = 32 - __clz(gmin ^ gmax);                  // bits [hi-1 .. 0] vary
+        pmask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
+        prefix = gmax & pmask;
+        bool use_cand = false;
+        int n_cand = 0;
+        for (int pass = 0; hi > 0; ++pass) {
+            const int wdt = min(8, hi), shift = hi - wdt, buf = pass & 1;
+            const uint32_t dmask = (1u << wdt) - 1u;
+            for (int i = tid; i < NW * 256; i += NT) whist[i >> 8][i & 255] = 0;
+            __syncthreads();
+            if (use_cand) {
+                for (int ci = tid; ci < n_cand; ci += NT) {
+                    const uint32_t key = bf.cand_key[ci];
+                    if ((key & pmask) == prefix) atomicAdd(&whist[wid][(key >> shift) & dmask], 1u);
+                }
+            } else {
+                for (int it = 0; it < seg; it += 32) {
+                    const int e = wid * seg + it + lane;
+                    if (e < cnt) {
+                        const uint32_t key = key_at(e);
+                        if ((key & pmask) == prefix) atomicAdd(&whist[wid][(key >> shift) & dmask], 1u);
+                    }
+                }
+            }
+            __syncthreads();
+            if (tid < 256) {
+                uint32_t t = 0;
+#pragma unroll 8
+                for (int w = 0; w < NW; ++w) t += whist[w][tid];
+                hist[buf][tid] = t;
+            }
+            __syncthreads();
+            csync();
+            // Cluster-wide count of bin 255 - tid, then counts of bins >= it.
+            uint32_t hv = 0;
+            if (tid < 256) {
+                uint32_t part[NC];
+#pragma unroll
+                for (int r = 0; r < NC; ++r) part[r] = remote(&hist[buf][0], r)[255 - tid];
+#pragma unroll
+                for (int r = 0; r < NC; ++r) hv += part[r];
+            }
+            const uint32_t incl = scan256(hv, scratch);
+            if (tid < 256 && incl >= krem && incl - hv < krem) {
+                s_digit = 255u - tid;
+                s_above = incl - hv;
+            }
+            __syncthreads();
+            prefix |= s_digit << shift;
+            pmask |= dmask << shift;
+            krem -= s_above;
+            hi = shift;
+            if (pass == 0 && hi > 0) {
+                // The keys of the threshold bin: usually a few hundred.
+                if (tid == 0) s_cnt[2] = 0;
+                __syncthreads();
+                for (int it = 0; it < seg; it += 32) {
+                    const int e = wid * seg + it + lane;
+                    const uint32_t key = e < cnt ? key_at(e) : 0u;
+                    const bool m = e < cnt && (key & pmask) == prefix;
+                    const uint32_t mb = __ballot_sync(0xffffffffu, m);
+                    uint32_t base = 0;
+                    if (lane == 0 && mb) base = atomicAdd(&s_cnt[2], (uint32_t)__popc(mb));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const uint32_t pos = base + __popc(mb & ((1u << lane) - 1u));
+                    if (m && pos < (uint32_t)CAND) {
+                        bf.cand_key[pos] = key;
+                        bf.cand_idx[pos] = (uint32_t)e;
+                    }
+                }
+                __syncthreads();
+                n_cand = (int)s_cnt[2];
+                use_cand = n_cand <= CAND;
+                // Cluster-wide candidate count.  An overflowing CTA reports
+                // CAND + 1: more than RANK_MAX in total, and the sum over the
+                // cluster cannot wrap.
+                static_assert(NC * (CAND + 1) < (1 << 30) && CAND + 1 > RANK_MAX, "candidate count encoding");
+                if (tid == 0) s_cnt[3] = use_cand ? (uint32_t)n_cand : (uint32_t)(CAND + 1);
+                csync();
+                uint32_t total = 0;
+                for (int r = 0; r < NC; ++r) total += remote(&s_cnt[3], r)[0];
+                // (the same decision in every CTA of the cluster)
+                if (total <= (uint32_t)RANK_MAX && chunk <= 32 * bf.bits_words) {
+                    // Rank every local candidate against all candidates of the cluster.
+                    const uint32_t *ak = bf.cand_key, *ai = nullptr;
+                    if constexpr (NC > 1) {
+                        uint32_t off = 0;
+                        for (int r = 0; r < NC; ++r) {
+                            const int nr = (int)remote(&s_cnt[3], r)[0];
+                            const uint32_t *rk = remote(bf.cand_key, r), *ri = remote(bf.cand_idx, r);
+                            for (int i = tid; i < nr; i += NT) {
+                                bf.all_key[off + i] = rk[i];
+                                bf.all_idx[off + i] = (uint32_t)(r * chunk) + ri[i];
+                            }
+                            off += (uint32_t)nr;
+                        }
+                        ak = bf.all_key;
+                        ai = bf.all_idx;
+                    }
+                    for (int i = tid; i < bf.bits_words; i += NT) bf.bits[i] = 0;
+                    __syncthreads();
+                    for (int ci = tid; ci < n_cand; ci += NT) {
+                        const uint32_t key = bf.cand_key[ci], li = bf.cand_idx[ci], gi = (uint32_t)lo + li;
+                        uint32_t above = 0;
+                        for (uint32_t j = 0; j < total; ++j) {
+                            const uint32_t kj = ak[j];
+                            const uint32_t ij = (NC > 1) ? ai[j] : (uint32_t)lo + bf.cand_idx[j];
+                            above += (kj > key) || (kj == key && ij < gi);
+                        }
+                        if (above < krem) atomicOr(&bf.bits[li >> 5], 1u << (li & 31));
+                    }
+                    __syncthreads();
+                    ranked = true;
+                    break;
+                }
+            }
+        }
+    }
+    // Selected: every key above the threshold bin (ranked) / key T (radix),
+    // plus the chosen keys of that bin (ranked: marked; radix: the first
+    // krem keys equal to T in index order).
+    const uint32_t T = prefix;
+    const uint32_t q_take = ranked ? 0xffffffffu : krem;
+    auto classify = [&](int e, bool valid, bool &g, bool &q) {
+        const uint32_t key = valid ? key_at(e) : 0u;
+        if (take_all) {
+            g = valid;
+            q = false;
+        } else if (ranked) {
+            const uint32_t top = key & pmask;
+            g = valid && top > T;
+            q = valid && top == T && ((bf.bits[e >> 5] >> (e & 31)) & 1u);
+        } else {
+            g = valid && key > T;
+            q = valid && key == T;
+        }
+    };
+    uint32_t ngt = 0, neq = 0;
+    for (int it = 0; it < seg; it += 32) {
+        const int e = wid * seg + it + lane;
+        bool g, q;
+        classify(e, e < cnt, g, q);
+        ngt += __popc(__ballot_sync(0xffffffffu, g));
+        neq += __popc(__ballot_sync(0xffffffffu, q));
+    }
+    if (lane == 0) {
+        wsum[wid][0] = ngt;
+        wsum[wid][1] = neq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t g = 0, q = 0;
+        for (int i = 0; i < NW; ++i) {
+            uint32_t a = wsum[i][0], bq = wsum[i][1];
+            wsum[i][0] = g;
+            wsum[i][1] = q;
+            g += a;
+            q += bq;
+        }
+        s_cnt[0] = g;
+        s_cnt[1] = q;
+    }
+    __syncthreads();
+    csync();
+    uint32_t gt_b = 0, eq_b = 0;
+    for (int r = 0; r < rank; ++r) {
+        const uint32_t *rc = remote(&s_cnt[0], r);
+        gt_b += rc[0];
+        eq_b += rc[1];
+    }
+    gt_b += wsum[wid][0];
+    eq_b += wsum[wid][1];
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int it = 0; it < seg; it += 32) {
+        const int e = wid * seg + it + lane;
+        const bool valid = e < cnt;
+        bool g, q;
+        classify(e, valid, g, q);
+        const uint32_t bg = __ballot_sync(0xffffffffu, g), bq = __ballot_sync(0xffffffffu, q);
+        const uint32_t my_gt = gt_b + __popc(bg & lt_mask), my_eq = eq_b + __popc(bq & lt_mask);
+        const int gi = lo + e;
+        const bool chosen = g || (q && my_eq < q_take);
+        if (chosen) {
+            const uint32_t pos = my_gt + min(my_eq, q_take);
+            if (o.expand) {
+                for (int j = 0; j < CSA2_BLOCK; ++j) {
+                    const int en = gi * CSA2_BLOCK + j;
+                    o.pool[(size_t)b * CSA2_POOL + pos * CSA2_BLOCK + j] = en < o.n_entries ? en : -1;
+                }
+            } else {
+                o.out[(size_t)b * o.out_stride + pos] = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
+            }
+        }
+        if (o.expand && valid && gi == n - 1)
+            o.pool_len[b] = kk * CSA2_BLOCK - (chosen ? n * CSA2_BLOCK - o.n_entries : 0);
+        gt_b += __popc(bg);
+        eq_b += __popc(bq);
+    }
+    if (rank == 0) {
+        if (o.expand) {
+            for (int i = kk * CSA2_BLOCK + tid; i < CSA2_POOL; i += NT) o.pool[(size_t)b * CSA2_POOL + i] = -1;
+            if (n == 0 && tid == 0) o.pool_len[b] = 0;
+        } else {
+            for (int i = kk + tid; i < k; i += NT) o.out[(size_t)b * o.out_stride + i] = -1;
+        }
+    }
+    // No CTA may leave while another still reads its shared memory.
+    csync();
+}
+
+}  // namespace sel
+}  // namespace csa2

@@ -16,9 +16,9 @@ from typing import List, Optional
 import torch
 
 import synth
-from . import (ATTEND_INPUTS_SETTLED, INDEX_FLAT, INDEX_FULL, INDEX_REINDEX, PAGE_CODES_BYTES, PAGE_ENTRIES, PAGE_KEYS_BYTES,
-               PAGE_SCALES_BYTES, PAGE_SUMM_BYTES, POOL, SWA_CODES_OFF, SWA_SCALE_OFF, TOPK, Cache, csa2_append,
-               csa2_attend, csa2_index, csa2_prefill, plane_offsets, workspace)
+from . import (ATTEND_INPUTS_SETTLED, INDEX_FLAT, INDEX_FULL, INDEX_REINDEX, KERNEL_ATTEND, PAGE_CODES_BYTES, PAGE_ENTRIES,
+               PAGE_KEYS_BYTES, PAGE_SCALES_BYTES, PAGE_SUMM_BYTES, POOL, SWA_CODES_OFF, SWA_SCALE_OFF, TOPK, Cache,
+               csa2_append, csa2_attend, csa2_index, csa2_prefill, csa2_set_profile_events, plane_offsets, workspace)
 
 SOFTMAX_SCALE = 1.0 / math.sqrt(512.0)
 PREFILL_CHUNK = 65536
@@ -70,7 +70,9 @@ class DeviceWorkload:
             self.cache.pending.copy_(self.saved_pending)
 
     # ------------------------------------------------------------ one step
-    def step(self, stream=None):
+    def step(self, stream=None, attend_events=None):
+        """One decode step.  attend_events = (layer, ev_start, ev_stop)
+        brackets that layer's attention launch with the two CUDA events."""
         w, c = self.w, self.cache
         if w.append:
             lat, key, gate, n_new = self.new
@@ -90,7 +92,12 @@ class DeviceWorkload:
             # A Reuse layer's indices were produced by its group's first layer,
             # not by the kernel right before it: its gather may start early.
             flags = ATTEND_INPUTS_SETTLED if mode == "reuse" else 0
+            timed = attend_events is not None and attend_events[0] == li
+            if timed:
+                csa2_set_profile_events(KERNEL_ATTEND, attend_events[1], attend_events[2])
             csa2_attend(c, q, self.topk[grp], SOFTMAX_SCALE, self.outs[li], self.ws, stream, flags=flags)
+            if timed:
+                csa2_set_profile_events(KERNEL_ATTEND, None, None)
 
     # ------------------------------------------------------------ read-back
     def entry_rows(self, b: int, entries: torch.Tensor):

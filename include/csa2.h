@@ -189,6 +189,18 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode,
                        int32_t *pool, int32_t *pool_len, int32_t *topk,
                        void *ws, size_t ws_bytes, csa2_stream_t stream);
 
+/* The indexer's selection step on its own ([blog-0539] §3: top_k 512 of the
+ * scored rows; top 2048 blocks in the hierarchical mode) ------------------
+ * For each row b < batch: the top min(k, n[b]) of scores[b*stride + 0 ..
+ * n[b]), score descending, ties to the lower index (-0 equals +0), written
+ * as indices in ascending order to out[b*k ..], -1 padded to k.
+ *   scores f32 device [batch][stride]; n int32 device [batch], each in
+ *   0..stride (values outside are clamped); k in 1..2048; out int32 device
+ *   [batch][k].  Scores must not be NaN.  Rows of up to 32768 elements are
+ *   selected by one CTA each, longer rows by an 8-CTA cluster.  No workspace. */
+csa2_status csa2_topk(const float *scores, int64_t stride, const int32_t *n, int32_t batch, int32_t k,
+                      int32_t *out, csa2_stream_t stream);
+
 /* Sparse MQA decode attention ([daiw] decode step and factor table: one
  * 512-dim latent shared by all heads, used as both K and V) --------------
  * For every head h of request b:
@@ -218,12 +230,14 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
  * framework that owns all device memory through its own pool and gives
  * plugins no way to allocate, or a serving loop that must not allocate once
  * it runs, because an allocation can synchronise the device.  It computes
- * exactly what csa2_attend computes, with the same arguments minus ws and
- * ws_bytes: the per-split partials live in one fixed array inside the
- * library instead of a caller workspace.
+ * what csa2_attend computes, with the same arguments minus ws, ws_bytes and
+ * flags, using the attention variant that exchanges its per-split partials
+ * through device memory: those partials live in one fixed array inside the
+ * library.  Results agree with csa2_attend up to the order of the final
+ * fp32 sum over the five splits.
  *   - Limit: batch * heads <= CSA2_ATTEND_NOALLOC_MAX_ROWS (512).  Larger
  *     calls return CSA2_ERR_UNSUPPORTED and enqueue nothing.
- *   - The array (512 x 10 x 514 floats, about 10.5 MB) exists on every GPU
+ *   - The array (512 x 5 x 512 floats, about 5.2 MB) exists on every GPU
  *     that loads the library and stays allocated until the process exits.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
@@ -245,7 +259,7 @@ typedef enum {
     CSA2_KERNEL_POOL_SCORE = 2,    /* FULL / REINDEX: exact pool rescoring     */
     CSA2_KERNEL_SELECT = 3,        /* radix top-k                              */
     CSA2_KERNEL_ATTEND = 4,        /* split-KV attention partials              */
-    CSA2_KERNEL_COMBINE = 5,       /* log-sum-exp combine                      */
+    CSA2_KERNEL_COMBINE = 5,       /* reserved: the merge runs inside ATTEND   */
     CSA2_KERNEL_COUNT = 6
 } csa2_kernel_id;
 

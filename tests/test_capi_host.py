@@ -79,5 +79,12 @@ def test_invalid_arguments_rejected_before_launch(csa2):
     assert L.csa2_prefill(C.byref(c), 0, 1, 0, 300, 300, good, good, good, None) == 1   # 4 pages = 256 entries
     assert L.csa2_attend(C.byref(c), 64, good, good, 0.1, good, 0, 6, good, 1 << 30, None) == 1   # unknown flag
     assert L.csa2_append(C.byref(c), None, good, good, good, None) == 1
+    # top-k: k out of 1..2048, null pointers, empty batch, zero stride
+    assert L.csa2_topk(good, 100, good, 4, 0, good, None) == 1
+    assert L.csa2_topk(good, 100, good, 4, 2049, good, None) == 1
+    assert L.csa2_topk(None, 100, good, 4, 512, good, None) == 1
+    assert L.csa2_topk(good, 100, None, 4, 512, good, None) == 1
+    assert L.csa2_topk(good, 100, good, 0, 512, good, None) == 1
+    assert L.csa2_topk(good, 0, good, 4, 512, good, None) == 1
     assert L.csa2_get_device_error(None, None, None) == 1
     assert csa2.status_string(1) == "invalid argument"

@@ -181,6 +181,63 @@ def test_sharp_softmax_variant():
     _check_step(w, dw, refs)
 
 
+def _exact_index_check(w, dw, refs):
+    """Every stage of the indexer against the oracle, index for index (the
+    crafted queries below make every score exact in fp32)."""
+    dw.step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    for b in range(w.batch):
+        ref = refs[b]
+        pool = dw.pool[b].cpu().numpy()
+        plen = int(dw.pool_len[b])
+        for li, mode in enumerate(w.layers):
+            if mode not in ("full", "reindex"):
+                continue
+            _, q_idx, hw = dw.layers[li]
+            qb, wb = bits(q_idx[b]), hw[b].cpu().numpy()
+            if mode == "full":
+                bs = oracle.score_f32(qb, wb, ref.summ)
+                rblocks = oracle.topk(bs, 2048)
+                rpool, rplen = oracle.expand_pool(rblocks, ref.n_entries)
+                assert plen == rplen and np.array_equal(pool, rpool), f"req {b}: pool"
+            rtop = oracle.index_pool(qb, wb, ref.keys8, pool, plen)
+            gtop = dw.topk[dw.layer_topk[li]][b].cpu().numpy()
+            assert np.array_equal(gtop, rtop), f"req {b} layer {li}: top-k"
+
+
+def test_index_ties_resolved_exactly():
+    """One-hot indexer queries: score = w * ReLU(+-key[d]) takes a few dozen
+    values, so thousands of blocks and entries tie; the tie rule (lower index
+    first) decides and must match the oracle exactly, through the block
+    selection, the pool and both the Full and the Reindex rescoring."""
+    w = synth.workload(3, small=True)
+    dw = DeviceWorkload(w, out_fp32=True)
+    for li, (d, h, sign, wt) in {0: (0, 0, 1.0, 1.0), 4: (5, 3, -1.0, 2.0)}.items():
+        q, q_idx, hw = dw.layers[li]
+        q_idx = torch.zeros_like(q_idx)
+        q_idx[:, h, d] = sign
+        hw = torch.zeros_like(hw)
+        hw[:, h] = wt
+        dw.layers[li] = (q, q_idx, hw)
+    refs = [OracleRequest(w, b, w.n_tok[b]) for b in range(w.batch)]
+    _exact_index_check(w, dw, refs)
+
+
+def test_index_all_scores_equal():
+    """A zero indexer query scores everything 0: the first 2048 blocks, the
+    first 16384 entries and then the first 512 of them are selected."""
+    w = synth.workload(3, small=True)
+    dw = DeviceWorkload(w, out_fp32=True)
+    for li in (0, 4):
+        q, q_idx, hw = dw.layers[li]
+        dw.layers[li] = (q, torch.zeros_like(q_idx), hw)
+    refs = [OracleRequest(w, b, w.n_tok[b]) for b in range(w.batch)]
+    _exact_index_check(w, dw, refs)
+    for b in range(w.batch):
+        assert np.array_equal(dw.topk[0][b].cpu().numpy(), np.arange(512))
+
+
 # ------------------------------------------------------------------ invariants
 def test_determinism_and_reuse_of_full_query():
     w = synth.workload(3, small=True)
