@@ -19,10 +19,16 @@ constexpr int IQ_PARTS = 3;
 constexpr int IQ_ROWS = IQ_PARTS * CSA2_IDX_HEADS;          // 96 rows: part p, head h at row 32p + h
 constexpr int IQ_BYTES = IQ_ROWS * CSA2_KEY_DIM;            // 12 KB of e5m2
 
-__device__ __forceinline__ float iq_e5m2_to_f32(uint8_t c)
+// An e5m2 code is the high byte of the fp16 with the same value.
+__device__ __forceinline__ float iq_e5m2_to_f32(uint32_t c) { return __half2float(__ushort_as_half((uint16_t)(c << 8))); }
+
+// x * 2^k, correctly rounded (as ldexpf) for k in [-126, 254]: a single
+// multiplication by an exact power of two when 2^k is a normal float, two
+// for k > 127 (both scale up, so neither rounds).
+__device__ __forceinline__ float iq_scale(float x, int k)
 {
-    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E5M2);
-    return __half2float(__half(h));
+    if (k <= 127) return x * __int_as_float((k + 127) << 23);
+    return (x * __int_as_float(254 << 23)) * __int_as_float((k - 127 + 127) << 23);
 }
 
 // Called by 128 threads (t = 0..127): head t/4, dims 32*(t%4) .. +31 of
@@ -50,14 +56,14 @@ __device__ __forceinline__ void iq_split(int t, const uint16_t *q_idx, const flo
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     int ex = 0;
     if (amax > 0.0f) frexpf(amax, &ex);
-    const int sh = (amax > 0.0f) ? 15 - ex : 0;              // amax * 2^sh in [2^14, 2^15)
+    const int sh = (amax > 0.0f) ? 15 - ex : 0;              // amax * 2^sh in [2^14, 2^15); sh in [-114, 164]
     uint32_t part[IQ_PARTS][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         uint32_t w0 = 0, w1 = 0, w2 = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            float r = ldexpf(x[4 * i + k], sh);
+            float r = iq_scale(x[4 * i + k], sh);
             const uint8_t c0 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);
             r -= iq_e5m2_to_f32(c0);
             const uint8_t c1 = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E5M2);

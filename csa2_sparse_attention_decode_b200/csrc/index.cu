@@ -16,7 +16,8 @@ namespace cg = cooperative_groups;
 namespace csa2 {
 
 // ------------------------------------------------------------------ top-k
-constexpr int SEL_CLUSTER = 8;         // CTAs per request (one thread-block cluster)
+// Rows longer than one CTA holds run on a cluster of 16 CTAs (8 where the
+// device cannot schedule 16 of these CTAs in one cluster).
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_CAP = 32768;         // keys a CTA keeps in shared memory (128 KB)
 constexpr int SEL_BITS = SEL_CAP / 32;
@@ -109,10 +110,10 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
         const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool, int32_t *pool_len
 #define CSA2_SELECT_PASS c, src, scores, score_stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len
 
-__global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREADS, 1)
-select_cluster_kernel(CSA2_SELECT_ARGS)
+template <int NC>
+__global__ void __launch_bounds__(SEL_THREADS, 1) select_cluster_kernel(CSA2_SELECT_ARGS)
 {
-    select_body<SEL_CLUSTER>(CSA2_SELECT_PASS);
+    select_body<NC>(CSA2_SELECT_PASS);
 }
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) select_cta_kernel(CSA2_SELECT_ARGS)
@@ -126,23 +127,36 @@ cudaError_t launch_select(const CacheView &c, int src, const float *scores, int6
                           int32_t *pool_len, int max_n, cudaStream_t st)
 {
     static bool attr_done[64] = {};
+    static int cluster_size[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const int smem = (int)SEL_SMEM;
     if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(select_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
+        const int nc = cluster_fits(select_cluster_kernel<16>, dim3(SEL_THREADS), smem, 16) ? 16 : 8;
+        if (dev < 64) {
+            cluster_size[dev] = nc;
+            attr_done[dev] = true;
+        }
     }
+    const int nc = dev < 64 ? cluster_size[dev] : 8;
     LaunchScope scope(CSA2_KERNEL_SELECT, st);
     if (max_n <= SEL_CAP)   // fits one CTA's shared memory: no cluster barriers on the path
         return launch_pdl(select_cta_kernel, dim3(1, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores, stride,
                           pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
-    return launch_pdl(select_cluster_kernel, dim3(SEL_CLUSTER, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores,
-                      stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
+    if (nc == 16)
+        return launch_pdl_cluster(select_cluster_kernel<16>, dim3(16, c.batch), dim3(SEL_THREADS), smem, st, 16, c,
+                                  src, scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
+    return launch_pdl_cluster(select_cluster_kernel<8>, dim3(8, c.batch), dim3(SEL_THREADS), smem, st, 8, c, src,
+                              scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
 }
 
 }  // namespace csa2

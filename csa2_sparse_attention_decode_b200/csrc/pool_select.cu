@@ -7,21 +7,23 @@
 // 2048 blocks x 8 positions = 16384 candidates; top_k 512; Full builds the
 // pool, Reindex searches inside it with its own query).
 //
-// One 8-CTA cluster per request.  CTA r scores pool rows [r*chunk,
-// r*chunk + chunk) (chunk a multiple of 128, at most 2048) and keeps the
+// One cluster of NC = 16 CTAs per request (8 where 16 cannot be scheduled).
+// CTA r scores pool rows [r*chunk, r*chunk + chunk) (chunk a multiple of
+// 128, at most 16384 / NC) and keeps the
 // order-preserving keys of its scores in shared memory; the cluster then runs
 // the selection of select.cuh over them and writes the selected pool ids.
 // Scoring roles (256 threads):
-//   warp 4      looks up the page of every 8-row run of the CTA's rows, then
-//               copies the runs (8 rows x 128 B of FP8 keys) by TMA into an
-//               8-stage ring of 128-row tiles, 128-byte swizzled;
-//   warp 5      issues the MMAs: D[128 x 32] (fp32, tensor memory) =
+//   warps 5-7   look up the page of every 8-row run of the CTA's rows, then
+//               copy the runs (8 rows x 128 B of FP8 keys) with 16-byte
+//               asynchronous copies into an 8-stage ring of 128-row tiles,
+//               128-byte swizzled;
+//   warp 4      issues the MMAs: D[128 x 32] (fp32, tensor memory) =
 //               sum_p K[128 x 128] (e4m3) . Qp^T (kind::f8f6f4), Q1 + Q2 + Q3
 //               the query split exactly into e5m2 parts (idx_query.cuh), into
 //               four rotating accumulators;
 //   warps 0-3   split the query, then one thread per row: score =
 //               sum_h w'_h ReLU(D[h]);
-//   warps 6-7   join for the selection.
+//   all warps then run the selection.
 #include <cudaTypedefs.h>
 
 #include <cooperative_groups.h>
@@ -39,22 +41,25 @@ using namespace umma;
 
 namespace {
 
-constexpr int NC = 8;                                    // CTAs per request
 constexpr int NT = 256;
 constexpr int TILE = 128;
 constexpr int STAGES = 8;
-constexpr int CHUNK_MAX = CSA2_POOL / NC;                // 2048 rows per CTA
-constexpr int RUNS = CHUNK_MAX / CSA2_BLOCK;             // 256 runs of 8 rows
+constexpr int NPROD = 96;                                // producer threads (warps 5-7)
 constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;         // 16 KB
-constexpr int RUN_BYTES = CSA2_BLOCK * CSA2_KEY_DIM;     // 1 KB
-constexpr int BITS_WORDS = CHUNK_MAX / 32;
-constexpr size_t OFF_Q = (size_t)STAGES * STAGE_BYTES;
-constexpr size_t OFF_KEYS = OFF_Q + IQ_BYTES;
-constexpr size_t OFF_CAND = OFF_KEYS + CHUNK_MAX * 4;
-constexpr size_t OFF_ALL = OFF_CAND + 2 * sel::CAND * 4;
-constexpr size_t OFF_BITS = OFF_ALL + 2 * sel::RANK_MAX * 4;
-constexpr size_t OFF_RUNS = OFF_BITS + BITS_WORDS * 4;
-constexpr size_t SMEM_BYTES = 1024 + OFF_RUNS + RUNS * 4;
+// Shared-memory layout for NC CTAs per request (rows per CTA at most POOL/NC).
+template <int NC>
+struct Layout {
+    static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 2048 (NC = 8) or 1024 (NC = 16) rows
+    static constexpr int RUNS = CHUNK_MAX / CSA2_BLOCK;  // runs of 8 rows
+    static constexpr int BITS_WORDS = CHUNK_MAX / 32;
+    static constexpr size_t OFF_Q = (size_t)STAGES * STAGE_BYTES;
+    static constexpr size_t OFF_KEYS = OFF_Q + IQ_BYTES;
+    static constexpr size_t OFF_CAND = OFF_KEYS + CHUNK_MAX * 4;
+    static constexpr size_t OFF_ALL = OFF_CAND + 2 * sel::CAND * 4;
+    static constexpr size_t OFF_BITS = OFF_ALL + 2 * sel::RANK_MAX * 4;
+    static constexpr size_t OFF_RUNS = OFF_BITS + BITS_WORDS * 4;
+    static constexpr size_t SMEM_BYTES = 1024 + OFF_RUNS + RUNS * 4;
+};
 constexpr int ACC = 4;                                   // accumulators in tensor memory
 constexpr int ACC_COLS = CSA2_IDX_HEADS;                 // 32 columns each
 constexpr int QPART_BYTES = CSA2_IDX_HEADS * CSA2_KEY_DIM;
@@ -82,16 +87,31 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
 }
 
 __device__ __forceinline__ void bar_workers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_producers() { asm volatile("bar.sync 2, 96;" ::: "memory"); }
 
-__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(NT, 1)
-pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const uint16_t *q_idx, const float *w,
-                   const int32_t *pool, const int32_t *pool_len, int32_t *topk)
+// 16-byte asynchronous global -> shared copy (L2 only), and an arrival on an
+// mbarrier once every copy this thread issued before it has landed (the
+// arrival counts towards the barrier's expected count).
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
 {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+template <int NC>
+__global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const uint16_t *q_idx, const float *w, const int32_t *pool, const int32_t *pool_len,
+                   int32_t *topk)
+{
+    using Lay = Layout<NC>;
+    constexpr int RUNS = Lay::RUNS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *ring = sm, *qbuf = sm + OFF_Q;
-    uint32_t *keys = reinterpret_cast<uint32_t *>(sm + OFF_KEYS);
-    int32_t *runs = reinterpret_cast<int32_t *>(sm + OFF_RUNS);
+    uint8_t *ring = sm, *qbuf = sm + Lay::OFF_Q;
+    uint32_t *keys = reinterpret_cast<uint32_t *>(sm + Lay::OFF_KEYS);
+    int32_t *runs = reinterpret_cast<int32_t *>(sm + Lay::OFF_RUNS);
     __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], d_full[ACC], d_empty[ACC], q_full;
     __shared__ float wq[CSA2_IDX_HEADS];
     __shared__ uint32_t tmem_base;
@@ -106,7 +126,7 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
     }
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], NPROD);
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < ACC; ++i) {
@@ -117,7 +137,6 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
         s_abort = 0;
         mbar_fence_init();
     }
-    if (tid == 32 * 4) tma_prefetch_map(&keys8);
     grid_dependency_wait();                      // the pool may come from the previous kernel
     allow_dependents();
     const int n_entries = n_entries_of(c, b);
@@ -132,26 +151,31 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
     volatile int *abort = &s_abort;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
 
-    if (warp == 4 && n_tiles > 0) {
-        // ------------------------------------------------------------ producer
-        // Plane row of every run: pool id, then page table, 8 runs per lane
-        // with all loads of a round in flight together.
+    if (warp >= 5 && n_tiles > 0) {
+        // ------------------------------------------------------------ producers
+        // Plane row of every run (pool id, then page table, each round's
+        // loads in flight together), then 16-byte asynchronous copies of the
+        // runs' rows into the ring, swizzled as the MMA reads them.  Gathered
+        // 1 KB runs are copied by the threads, not by TMA: a tile is 16 runs
+        // from unrelated pages.
+        const int ptid = tid - 5 * 32;
         const int n_runs = (cnt + CSA2_BLOCK - 1) / CSA2_BLOCK;
-        int e_[8], pg_[8];
+        constexpr int RPT = (RUNS + NPROD - 1) / NPROD;          // runs per producer thread
+        int e_[RPT], pg_[RPT];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = lane + 32 * u;
+        for (int u = 0; u < RPT; ++u) {
+            const int j = ptid + NPROD * u;
             e_[u] = j < n_runs ? pool[(size_t)b * CSA2_POOL + lo + CSA2_BLOCK * j] : -1;
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < RPT; ++u) {
             const int e = e_[u];
             pg_[u] = (e >= 0 && e < n_entries && (e >> 6) < c.max_pages)
                          ? c.page_table[(size_t)b * c.max_pages + (e >> 6)] : -1;
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = lane + 32 * u;
+        for (int u = 0; u < RPT; ++u) {
+            const int j = ptid + NPROD * u;
             if (j >= n_runs) continue;
             const int e = e_[u], pg = pg_[u];
             int pid = -1;
@@ -161,27 +185,32 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
             else pid = pg * CSA2_PAGE_ENTRIES + (e & (CSA2_PAGE_ENTRIES - 1));
             runs[j] = pid;
         }
-        __syncwarp();
+        bar_producers();
         int issued = 0;
         for (int t = 0; t < n_tiles; ++t) {
             const int s = t % STAGES;
             bool okw = true;
             if (lane == 0 && t >= STAGES) okw = wait_or_abort(&empty[s], ((t / STAGES) - 1) & 1, abort, c.error);
             if (!__shfl_sync(0xffffffffu, okw, 0)) break;          // warp-uniform decision
-            const int j = 16 * t + lane;
-            const int row = (lane < 16 && j < n_runs) ? runs[j] : -1;
-            const uint32_t ok = __ballot_sync(0xffffffffu, row >= 0);
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)__popc(ok) * RUN_BYTES);
-            __syncwarp();
-            if (row >= 0) tma_load_2d(ring + s * STAGE_BYTES + lane * RUN_BYTES, &keys8, 0, row, &full[s]);
-            __syncwarp();
+            uint8_t *stage = ring + s * STAGE_BYTES;
+            // 16 runs x 8 rows x 8 chunks of 16 bytes
+            for (int i = ptid; i < TILE * 8; i += NPROD) {
+                const int run = 16 * t + (i >> 6), r8 = (i >> 3) & 7, ch = i & 7;
+                const int pid = run < n_runs ? runs[run] : -1;
+                if (pid >= 0) {
+                    const int row = ((i >> 6) << 3) + r8;
+                    cp_async16(stage + row * 128 + ((ch ^ (row & 7)) << 4),
+                               c.keys + (size_t)(pid + r8) * CSA2_KEY_DIM + ch * 16);
+                }
+            }
+            cp_async_arrive(&full[s]);                              // one arrival per thread, when its copies land
             issued = t + 1;
         }
         // Never leave with copies in flight: wait for the last stages to land.
         if (lane == 0)
             for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
         __syncwarp();
-    } else if (warp == 5 && n_tiles > 0) {
+    } else if (warp == 4 && n_tiles > 0) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t qaddr = smem_addr(qbuf);
         int issued = 0;
@@ -196,6 +225,7 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
             if (!__shfl_sync(0xffffffffu, okw, 0)) break;          // warp-uniform decision
             fence_after_sync();
             if (lane == 0) {
+                fence_proxy_async_smem();                           // the copies were generic-proxy writes
                 const uint32_t aaddr = smem_addr(ring + s * STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < CSA2_KEY_DIM / 32; ++kk)
@@ -253,12 +283,12 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
     sel::Bufs bf;
     bf.keys = keys;
     bf.scores = nullptr;
-    bf.cand_key = reinterpret_cast<uint32_t *>(sm + OFF_CAND);
+    bf.cand_key = reinterpret_cast<uint32_t *>(sm + Lay::OFF_CAND);
     bf.cand_idx = bf.cand_key + sel::CAND;
-    bf.all_key = reinterpret_cast<uint32_t *>(sm + OFF_ALL);
+    bf.all_key = reinterpret_cast<uint32_t *>(sm + Lay::OFF_ALL);
     bf.all_idx = bf.all_key + sel::RANK_MAX;
-    bf.bits = reinterpret_cast<uint32_t *>(sm + OFF_BITS);
-    bf.bits_words = BITS_WORDS;
+    bf.bits = reinterpret_cast<uint32_t *>(sm + Lay::OFF_BITS);
+    bf.bits_words = Lay::BITS_WORDS;
     sel::Out o;
     o.out = topk;
     o.out_stride = CSA2_TOPK;
@@ -277,40 +307,40 @@ pool_select_kernel(const __grid_constant__ CUtensorMap keys8, CacheView c, const
     }
 }
 
-// 2-D byte tensor over the key plane: rows of 128 bytes, boxes of 8 rows,
-// 128-byte swizzled.
-bool make_keys8_map(CUtensorMap *m, void *base, long long rows)
-{
-    auto fn = tensor_map_encoder();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {128, (cuuint32_t)CSA2_BLOCK};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const float *w, const int32_t *pool,
                                const int32_t *pool_len, int32_t *topk, cudaStream_t st)
 {
+    // 16 CTAs per request where the device can schedule such clusters
+    // (shorter per-CTA row ranges), else 8.
     static bool attr_done[64] = {};
+    static int cluster_size[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(pool_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        e = cudaFuncSetAttribute(pool_select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Layout<8>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)Layout<16>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
+        const int nc = cluster_fits(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16) ? 16 : 8;
+        if (dev < 64) {
+            cluster_size[dev] = nc;
+            attr_done[dev] = true;
+        }
     }
-    CUtensorMap keys8;
-    if (!make_keys8_map(&keys8, c.keys, (long long)c.n_pages * CSA2_PAGE_ENTRIES)) return cudaErrorInvalidValue;
+    const int nc = dev < 64 ? cluster_size[dev] : 8;
     LaunchScope scope(CSA2_KERNEL_POOL_SCORE, st);
-    return launch_pdl(pool_select_kernel, dim3(NC, c.batch), dim3(NT), SMEM_BYTES, st, keys8, c, q_idx, w, pool,
-                      pool_len, topk);
+    if (nc == 16)
+        return launch_pdl_cluster(pool_select_kernel<16>, dim3(16, c.batch), dim3(NT), Layout<16>::SMEM_BYTES, st, 16,
+                                  c, q_idx, w, pool, pool_len, topk);
+    return launch_pdl_cluster(pool_select_kernel<8>, dim3(8, c.batch), dim3(NT), Layout<8>::SMEM_BYTES, st, 8, c,
+                              q_idx, w, pool, pool_len, topk);
 }
 
 }  // namespace csa2

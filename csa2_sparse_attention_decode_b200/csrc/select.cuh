@@ -9,9 +9,9 @@
 //   2. one 8-bit histogram pass over the next bits finds the bin that holds
 //      the k-th largest key and how many keys of that bin to take (krem);
 //   3. the keys of that bin (the candidates, usually a few hundred) are
-//      compacted.  When the cluster holds at most RANK_MAX of them, each
-//      candidate is ranked directly against all candidates (key desc, index
-//      asc) and marked when its rank is below krem.  Otherwise further 8-bit
+//      compacted.  When the cluster holds few enough of them, each candidate
+//      is ranked directly (one warp per candidate) against all candidates
+//      (key desc, index asc) and marked when its rank is below krem.  Otherwise further 8-bit
 //      passes over the candidates (or all keys, if they overflowed) find the
 //      exact threshold key T, and the first krem keys equal to T in index
 //      order are taken;
@@ -31,6 +31,7 @@ namespace cg = cooperative_groups;
 
 constexpr int CAND = 2048;       // candidates a CTA keeps after the first pass
 constexpr int RANK_MAX = 2048;   // cluster-wide candidates ranked directly
+constexpr uint32_t RANK_WORK = 1024;   // at most this many comparisons per lane
 
 // Order-preserving 32-bit key of an fp32 score (-0 folded onto +0).
 __device__ __forceinline__ uint32_t ord_key(float x)
@@ -81,9 +82,9 @@ __device__ __forceinline__ uint32_t scan256(uint32_t v, uint32_t *scratch)
 
 // Selects the top min(k, n) of the n elements of request b; CTA r of the NC
 // holds elements [r*chunk, r*chunk + chunk) of them, this one [lo, lo + cnt)
-// with lo = rank*chunk.  kmin / kmax: this thread's
-// min / max over the keys it staged (any split of the range over the
-// threads).  NT = threads per CTA (a multiple of 32, at least 256).
+// with lo = rank*chunk.  kmin / kmax: this thread's min / max over the keys
+// it staged (any split of the range over the threads; a thread without keys
+// passes kmin = 0xffffffff, kmax = 0).  NT = threads per CTA (a multiple of 32, at least 256).
 template <int NC, int NT>
 __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int chunk, int lo, int cnt, int k,
                                             uint32_t kmin, uint32_t kmax, const Out &o)
@@ -92,8 +93,11 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     __shared__ uint32_t hist[2][256];
     __shared__ uint32_t whist[NW][256];
     __shared__ uint32_t scratch[32];
-    __shared__ uint32_t wsum[NW][2];
+    __shared__ uint32_t wsum[NW][4];
     __shared__ uint32_t s_cnt[4];
+    __shared__ uint32_t s_mm[4];
+    __shared__ uint32_t s_rk[NC][4];                       // per-rank values gathered by warp 0
+
     __shared__ uint32_t s_digit, s_above;
     const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
     auto csync = [&]() {
@@ -105,6 +109,16 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         else return ptr;
     };
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    // Warp 0 reads word(s) src[0..nw) of every CTA of the cluster into
+    // s_rk[rank][..]; everyone else reads them from there (remote loads stay
+    // NC * nw per CTA instead of per thread).
+    auto gather_ranks = [&](uint32_t *src, int nw) {
+        if (wid == 0 && lane < NC) {
+            const uint32_t *rc = remote(src, lane);
+            for (int i = 0; i < nw; ++i) s_rk[lane][i] = rc[i];
+        }
+        __syncthreads();
+    };
     const int kk = min(k, n);
     const bool take_all = n <= k;
     const int seg = ((cnt + NW * 32 - 1) / (NW * 32)) * 32;     // elements per warp, multiple of 32
@@ -113,33 +127,50 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kk;
     bool ranked = false;                                    // candidates were ranked directly
     if (!take_all) {
+        // Range of the keys that matter.  Every thread holding a key holds
+        // one >= its own maximum, so when at least kk threads hold keys, the
+        // smallest per-thread maximum lb is a lower bound of the threshold:
+        // keys below it never need resolving, however far below they lie.
+        const bool has = kmin <= kmax;
+        uint32_t klb = has ? kmax : 0xffffffffu;
+        uint32_t nthr = __popc(__ballot_sync(0xffffffffu, has));
 #pragma unroll
         for (int off = 16; off; off >>= 1) {
             kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
             kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+            klb = min(klb, __shfl_xor_sync(0xffffffffu, klb, off));
         }
         if (lane == 0) {
             wsum[wid][0] = kmin;
             wsum[wid][1] = kmax;
+            wsum[wid][2] = klb;
+            wsum[wid][3] = nthr;
         }
         __syncthreads();
         if (tid == 0) {
-            uint32_t a = 0xffffffffu, z = 0u;
+            uint32_t a = 0xffffffffu, z = 0u, l = 0xffffffffu, t = 0u;
             for (int i = 0; i < NW; ++i) {
                 a = min(a, wsum[i][0]);
                 z = max(z, wsum[i][1]);
+                l = min(l, wsum[i][2]);
+                t += wsum[i][3];
             }
-            s_cnt[0] = a;
-            s_cnt[1] = z;
+            s_mm[0] = a;
+            s_mm[1] = z;
+            s_mm[2] = l;
+            s_mm[3] = t;
         }
         csync();
-        uint32_t gmin = 0xffffffffu, gmax = 0u;
+        gather_ranks(&s_mm[0], 4);
+        uint32_t gmin = 0xffffffffu, gmax = 0u, glb = 0xffffffffu, gthr = 0u;
         for (int r = 0; r < NC; ++r) {
-            const uint32_t *rc = remote(&s_cnt[0], r);
-            gmin = min(gmin, rc[0]);
-            gmax = max(gmax, rc[1]);
+            gmin = min(gmin, s_rk[r][0]);
+            gmax = max(gmax, s_rk[r][1]);
+            glb = min(glb, s_rk[r][2]);
+            gthr += s_rk[r][3];
         }
-        int hi = 32 - __clz(gmin ^ gmax);                  // bits [hi-1 .. 0] vary
+        const uint32_t low = gthr >= (uint32_t)kk ? glb : gmin;
+        int hi = 32 - __clz(low ^ gmax);                    // bits [hi-1 .. 0] vary above `low`
         pmask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
         prefix = gmax & pmask;
         bool use_cand = false;
@@ -218,37 +249,47 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
                 static_assert(NC * (CAND + 1) < (1 << 30) && CAND + 1 > RANK_MAX, "candidate count encoding");
                 if (tid == 0) s_cnt[3] = use_cand ? (uint32_t)n_cand : (uint32_t)(CAND + 1);
                 csync();
-                uint32_t total = 0;
-                for (int r = 0; r < NC; ++r) total += remote(&s_cnt[3], r)[0];
-                // (the same decision in every CTA of the cluster)
-                if (total <= (uint32_t)RANK_MAX && chunk <= 32 * bf.bits_words) {
+                __syncthreads();                            // s_rk is reused
+                gather_ranks(&s_cnt[3], 1);
+                uint32_t total = 0, most = 0;
+                for (int r = 0; r < NC; ++r) {
+                    const uint32_t v = s_rk[r][0];
+                    total += v;
+                    most = max(most, v);
+                }
+                // Rank directly when the comparisons per lane stay small (the
+                // same decision in every CTA of the cluster).
+                const uint32_t work = ((most + NW - 1) / NW) * ((total + 31) / 32);
+                if (total <= (uint32_t)RANK_MAX && work <= RANK_WORK && chunk <= 32 * bf.bits_words) {
                     // Rank every local candidate against all candidates of the cluster.
                     const uint32_t *ak = bf.cand_key, *ai = nullptr;
                     if constexpr (NC > 1) {
-                        uint32_t off = 0;
-                        for (int r = 0; r < NC; ++r) {
-                            const int nr = (int)remote(&s_cnt[3], r)[0];
-                            const uint32_t *rk = remote(bf.cand_key, r), *ri = remote(bf.cand_idx, r);
-                            for (int i = tid; i < nr; i += NT) {
-                                bf.all_key[off + i] = rk[i];
-                                bf.all_idx[off + i] = (uint32_t)(r * chunk) + ri[i];
-                            }
-                            off += (uint32_t)nr;
+                        // Candidate g of the cluster: CTA r's number g - off[r]
+                        // (all remote loads independent of one another).
+                        for (uint32_t g = tid; g < total; g += NT) {
+                            int r = 0;
+                            uint32_t off = 0;
+                            while (r < NC - 1 && g >= off + s_rk[r][0]) off += s_rk[r++][0];
+                            const uint32_t i = g - off;
+                            bf.all_key[g] = remote(bf.cand_key, r)[i];
+                            bf.all_idx[g] = (uint32_t)(r * chunk) + remote(bf.cand_idx, r)[i];
                         }
                         ak = bf.all_key;
                         ai = bf.all_idx;
                     }
                     for (int i = tid; i < bf.bits_words; i += NT) bf.bits[i] = 0;
                     __syncthreads();
-                    for (int ci = tid; ci < n_cand; ci += NT) {
+                    // One warp per local candidate; its lanes split the comparisons.
+                    for (int ci = wid; ci < n_cand; ci += NW) {
                         const uint32_t key = bf.cand_key[ci], li = bf.cand_idx[ci], gi = (uint32_t)lo + li;
                         uint32_t above = 0;
-                        for (uint32_t j = 0; j < total; ++j) {
+                        for (uint32_t j = lane; j < total; j += 32) {
                             const uint32_t kj = ak[j];
                             const uint32_t ij = (NC > 1) ? ai[j] : (uint32_t)lo + bf.cand_idx[j];
                             above += (kj > key) || (kj == key && ij < gi);
                         }
-                        if (above < krem) atomicOr(&bf.bits[li >> 5], 1u << (li & 31));
+                        above = __reduce_add_sync(0xffffffffu, above);
+                        if (lane == 0 && above < krem) atomicOr(&bf.bits[li >> 5], 1u << (li & 31));
                     }
                     __syncthreads();
                     ranked = true;
@@ -303,11 +344,11 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     }
     __syncthreads();
     csync();
+    gather_ranks(&s_cnt[0], 2);
     uint32_t gt_b = 0, eq_b = 0;
     for (int r = 0; r < rank; ++r) {
-        const uint32_t *rc = remote(&s_cnt[0], r);
-        gt_b += rc[0];
-        eq_b += rc[1];
+        gt_b += s_rk[r][0];
+        eq_b += s_rk[r][1];
     }
     gt_b += wsum[wid][0];
     eq_b += wsum[wid][1];
