@@ -219,7 +219,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     if (tid == 0) {
         mbar_init(&bar_q, 1);
         mbar_init(&bar_s, 1);
-        mbar_init(&bar_o, 1);
+        mbar_init(&bar_o, 4);                                // one commit per issuing warp
         mbar_fence_init();
         // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x 32 heads, 128-byte
         // swizzled (K-major operand layout); heads past `heads` read as zero.
@@ -295,10 +295,12 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         fence_proxy_async_smem();
         __syncthreads();
         fence_after_sync();
-        // ---- 5. O^T = V^T . P^T (hi, then lo), 128 dims per chunk
-        if (tid == 0) {
+        // ---- 5. O^T = V^T . P^T (hi, then lo), 128 dims per chunk; lane 0 of
+        // warp cc issues chunk cc (four issuers, disjoint accumulators)
+        if (lane == 0 && warp < 4) {
             const uint32_t va = smem_addr(Vs), ph = smem_addr(Ph), pl = smem_addr(Pl);
-            for (int cc = 0; cc < 4; ++cc) {
+            const int cc = warp;
+            {
                 for (int part = 0; part < 2; ++part) {
                     const uint32_t pb = part ? pl : ph;
 #pragma unroll
