@@ -358,17 +358,29 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     }
     cluster.sync();                                       // partials visible cluster-wide
     {
+        // This CTA's fifth (at most 820 float4, two per thread): every remote
+        // load of both is issued before any sum.
         constexpr int total4 = HG * (CSA2_LATENT / 4);
+        static_assert((total4 + NTILES - 1) / NTILES <= 2 * THREADS, "two outputs per thread");
         const int lo4 = tile * total4 / NTILES, hi4 = (tile + 1) * total4 / NTILES;
-        for (int i = lo4 + tid; i < hi4; i += THREADS) {
-            const int hh = i / (CSA2_LATENT / 4), d4 = i % (CSA2_LATENT / 4);
-            if (hh >= nh) continue;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 v[2][NTILES];
 #pragma unroll
-            for (int r = 0; r < NTILES; ++r) {
-                if (!tile_live[r]) continue;
-                const float4 v = reinterpret_cast<const float4 *>(cluster.map_shared_rank(Ob, r))[i];
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        for (int u = 0; u < 2; ++u) {
+            const int i = lo4 + tid + u * THREADS;
+#pragma unroll
+            for (int r = 0; r < NTILES; ++r)
+                v[u][r] = (i < hi4 && tile_live[r]) ? reinterpret_cast<const float4 *>(cluster.map_shared_rank(Ob, r))[i]
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = lo4 + tid + u * THREADS;
+            const int hh = i / (CSA2_LATENT / 4), d4 = i % (CSA2_LATENT / 4);
+            if (i >= hi4 || hh >= nh) continue;
+            float4 acc = v[u][0];
+#pragma unroll
+            for (int r = 1; r < NTILES; ++r) {
+                acc.x += v[u][r].x; acc.y += v[u][r].y; acc.z += v[u][r].z; acc.w += v[u][r].w;
             }
             const size_t o = ((size_t)b * heads + hg0 + hh) * CSA2_LATENT + 4 * d4;
             if (out_is_fp32) {

@@ -34,7 +34,7 @@ using namespace umma;
 namespace {
 
 constexpr int TILE = 128;
-constexpr int STAGES = 6;
+constexpr int STAGES = 4;
 constexpr int CTAS_PER_SM = 2;                              // two independent pipelines per SM
 constexpr int PW = 16;                                      // producer look-up window (tiles)
 constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;            // 16 KB

@@ -15,7 +15,10 @@
 //      passes over the candidates (or all keys, if they overflowed) find the
 //      exact threshold key T, and the first krem keys equal to T in index
 //      order are taken;
-//   4. a counting pass and an ordered compaction write the selected ids.
+//   4. the selected ids are written in ascending order: when every decision
+//      is local (ranked candidates, or all elements taken) one pass compacts
+//      each warp's selections in place; otherwise (ties at T resolved in
+//      index order) a counting pass precedes the ordered compaction.
 // Histograms, counts and candidates are exchanged over distributed shared
 // memory.  Used by the top-k kernels of index.cu and by the fused pool
 // rescoring kernel.
@@ -43,7 +46,7 @@ __device__ __forceinline__ uint32_t ord_key(float x)
 
 // Shared-memory work areas the caller provides (dynamic shared memory).
 struct Bufs {
-    const uint32_t *keys;        // [cnt] keys of this CTA's range, or nullptr: read `scores`
+    uint32_t *keys;              // [cnt] keys of this CTA's range, or nullptr: read `scores`
     const float *scores;         // global scores of this CTA's range (when keys == nullptr)
     uint32_t *cand_key, *cand_idx;    // [CAND]
     uint32_t *all_key, *all_idx;      // [RANK_MAX]
@@ -317,6 +320,67 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
             q = valid && key == T;
         }
     };
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    auto write_one = [&](int gi, uint32_t pos) {
+        if (o.expand) {
+            for (int j = 0; j < CSA2_BLOCK; ++j) {
+                const int en = gi * CSA2_BLOCK + j;
+                o.pool[(size_t)b * CSA2_POOL + pos * CSA2_BLOCK + j] = en < o.n_entries ? en : -1;
+            }
+        } else {
+            o.out[(size_t)b * o.out_stride + pos] = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
+        }
+    };
+    auto pad_tail = [&]() {
+        if (rank == 0) {
+            if (o.expand) {
+                for (int i = kk * CSA2_BLOCK + tid; i < CSA2_POOL; i += NT) o.pool[(size_t)b * CSA2_POOL + i] = -1;
+                if (n == 0 && tid == 0) o.pool_len[b] = 0;
+            } else {
+                for (int i = kk + tid; i < k; i += NT) o.out[(size_t)b * o.out_stride + i] = -1;
+            }
+        }
+    };
+    if ((ranked || take_all) && bf.keys) {
+        // Every decision is local: one pass compacts each warp's chosen
+        // elements in place (over keys it has already read), then the
+        // warps' and CTAs' counts place them.
+        uint32_t c = 0;
+        for (int it = 0; it < seg; it += 32) {
+            const int e = wid * seg + it + lane;
+            const bool valid = e < cnt;
+            bool g, q;
+            classify(e, valid, g, q);
+            const bool chosen = g || q;
+            const uint32_t bal = __ballot_sync(0xffffffffu, chosen);
+            if (chosen) bf.keys[wid * seg + c + __popc(bal & lt_mask)] = (uint32_t)e;
+            c += __popc(bal);
+            if (o.expand && valid && lo + e == n - 1)
+                o.pool_len[b] = kk * CSA2_BLOCK - (chosen ? n * CSA2_BLOCK - o.n_entries : 0);
+        }
+        if (lane == 0) wsum[wid][1] = c;
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t a = 0;
+            for (int i = 0; i < NW; ++i) {
+                wsum[i][0] = a;
+                a += wsum[i][1];
+            }
+            s_cnt[0] = a;
+        }
+        __syncthreads();
+        csync();
+        gather_ranks(&s_cnt[0], 1);
+        uint32_t base = wsum[wid][0];
+        for (int r = 0; r < rank; ++r) base += s_rk[r][0];
+        // Nobody reads this CTA's shared memory after this point.
+        if constexpr (NC > 1) asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
+        const uint32_t nw = wsum[wid][1];
+        for (uint32_t j = lane; j < nw; j += 32) write_one(lo + (int)bf.keys[wid * seg + j], base + j);
+        pad_tail();
+        if constexpr (NC > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+        return;
+    }
     uint32_t ngt = 0, neq = 0;
     for (int it = 0; it < seg; it += 32) {
         const int e = wid * seg + it + lane;
@@ -352,7 +416,6 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     }
     gt_b += wsum[wid][0];
     eq_b += wsum[wid][1];
-    const uint32_t lt_mask = (1u << lane) - 1u;
     for (int it = 0; it < seg; it += 32) {
         const int e = wid * seg + it + lane;
         const bool valid = e < cnt;
@@ -362,30 +425,13 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         const uint32_t my_gt = gt_b + __popc(bg & lt_mask), my_eq = eq_b + __popc(bq & lt_mask);
         const int gi = lo + e;
         const bool chosen = g || (q && my_eq < q_take);
-        if (chosen) {
-            const uint32_t pos = my_gt + min(my_eq, q_take);
-            if (o.expand) {
-                for (int j = 0; j < CSA2_BLOCK; ++j) {
-                    const int en = gi * CSA2_BLOCK + j;
-                    o.pool[(size_t)b * CSA2_POOL + pos * CSA2_BLOCK + j] = en < o.n_entries ? en : -1;
-                }
-            } else {
-                o.out[(size_t)b * o.out_stride + pos] = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
-            }
-        }
+        if (chosen) write_one(gi, my_gt + min(my_eq, q_take));
         if (o.expand && valid && gi == n - 1)
             o.pool_len[b] = kk * CSA2_BLOCK - (chosen ? n * CSA2_BLOCK - o.n_entries : 0);
         gt_b += __popc(bg);
         eq_b += __popc(bq);
     }
-    if (rank == 0) {
-        if (o.expand) {
-            for (int i = kk * CSA2_BLOCK + tid; i < CSA2_POOL; i += NT) o.pool[(size_t)b * CSA2_POOL + i] = -1;
-            if (n == 0 && tid == 0) o.pool_len[b] = 0;
-        } else {
-            for (int i = kk + tid; i < k; i += NT) o.out[(size_t)b * o.out_stride + i] = -1;
-        }
-    }
+    pad_tail();
     // No CTA may leave while another still reads its shared memory.
     csync();
 }
