@@ -4,7 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference] [--config C]
 
 One step = the whole decode hot path over one batch: (append,) index and the
-attends of every layer of the workload's schedule.  Default workload: the
+attends of every layer of the workload's schedule.  --config 5 runs the
+40-layer whole-model schedule (several caches) instead.  Default workload: the
 reuse group at 1M context (4 requests x 1,048,576 entries, Full + 3 Reuse +
 Reindex + 3 Reuse, 64 heads).  The step is captured once in a CUDA graph and
 replayed; each timed replay is bracketed by CUDA events, with a 256 MB write
@@ -59,10 +60,12 @@ def job_throughput(world: int, batch_per_rank: int, steps: int, max_total_ms: fl
 
 def algorithmic_bytes(w: synth.Workload) -> dict:
     """Bytes the step must move, per the layout (per request, summed):
-    index  FULL: ceil(N/8)*128 [if > 2048 blocks] + min(N,16384)*128 + 16384*4
-           FLAT: N*128;  REINDEX: 16384*(128+4)
-    attend per layer: 512*288 + min(n_tok,128)*516 + 2*H*512*2 + 512*4
-    append: m*(641)*4 + 416 + 128 + 7*128 + m*516."""
+    index  FULL: ceil(N/8)*128 [if > 2048 blocks] + min(N,16384)*(128+4)
+           FLAT: N*128;  REINDEX: min(N,16384)*(128+4)
+    attend per layer: 512*288 + 512*4 (top-k rows, not for SWA-only layers)
+                      + min(n_tok,128)*516 + 2*H*512*2
+    append per new token: 641*4 in + 516 SWA; per completed entry: 416 + 128
+                      summary + 7*128 keys re-read."""
     tot = {"index": 0, "block_summaries": 0, "attend": 0, "append": 0}
     for b in range(w.batch):
         T = w.n_tok[b] + w.n_new[b]
@@ -74,15 +77,25 @@ def algorithmic_bytes(w: synth.Workload) -> dict:
                     tot["index"] += N * 128
                 else:
                     summ = nb * 128 if nb > 2048 else 0
-                    tot["block_summaries"] += nb * 128
-                    tot["index"] += summ + min(N, 16384) * 128 + 16384 * 4
+                    tot["block_summaries"] += summ
+                    tot["index"] += summ + min(N, 16384) * (128 + 4)
             elif mode == "reindex":
-                tot["index"] += 16384 * (128 + 4)
-            tot["attend"] += 512 * 288 + min(T, 128) * 516 + 2 * w.heads * 512 * 2 + 512 * 4
+                tot["index"] += min(N, 16384) * (128 + 4)
+            window = min(T, 128) * 516 + 2 * w.heads * 512 * 2
+            tot["attend"] += window + (0 if mode == "swa" else 512 * 288 + 512 * 4)
         if w.append:
-            m = w.m[b]
-            tot["append"] += m * 641 * 4 + 416 + 128 + 7 * 128 + m * 516
+            new_entries = T // w.m[b] - w.n_tok[b] // w.m[b]
+            tot["append"] += w.n_new[b] * (641 * 4 + 516) + new_entries * (416 + 128 + 7 * 128)
     tot["step"] = tot["index"] + tot["attend"] + tot["append"]
+    return tot
+
+
+def schedule_bytes(ws) -> dict:
+    """algorithmic_bytes summed over the caches of a schedule."""
+    tot = {}
+    for w in ws:
+        for k, v in algorithmic_bytes(w).items():
+            tot[k] = tot.get(k, 0) + v
     return tot
 
 
@@ -299,25 +312,78 @@ def run_reference(args, w: synth.Workload, rank: int, world: int):
 
 
 # ------------------------------------------------------------------ GPU side
-def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
+class Runner:
+    """What the timed loop drives: one cache's DeviceWorkload (configs 0-4)
+    or the 40-layer whole-model schedule of several caches (config 5)."""
+
+    def __init__(self, args, dev):
+        from csa2_sparse_attention_decode_b200.harness import DeviceWorkload, ScheduleWorkload
+        if args.config == 5:
+            sched = synth.schedule40(args.small)
+            sw = ScheduleWorkload(sched, dev)
+            self.name, self.ws, self.parts, self.step = sched.name, list(sched.caches), sw.parts, sw.step
+            self.kv_bytes_per_token = sched.kv_bytes_per_token()
+        else:
+            w = synth.workload(args.config, args.small)
+            dw = DeviceWorkload(w, dev)
+            self.name, self.ws, self.parts, self.step = w.name, [w], [dw], dw.step
+            self.kv_bytes_per_token = None
+        self.batch = self.ws[0].batch
+        self.n_layers = sum(len(w.layers) for w in self.ws)
+        self.append = any(w.append for w in self.ws)
+        self.flat = any(w.index == "flat" for w in self.ws)
+
+    def restore(self, stream):
+        for p in self.parts:
+            p.restore(stream)
+
+    def inputs(self):
+        """Device tensors a caller provides per step: every layer's q, the
+        indexer q / w of Full and Reindex layers, and the appended tokens."""
+        ins = []
+        for p in self.parts:
+            for li, mode in enumerate(p.w.layers):
+                ins.append(p.layers[li][0])
+                if mode in ("full", "reindex"):
+                    ins += [p.layers[li][1], p.layers[li][2]]
+            if p.w.append:
+                ins += list(p.new)
+        return ins
+
+    def outs(self):
+        return [o for p in self.parts for o in p.outs]
+
+    def config(self) -> dict:
+        if len(self.ws) == 1:
+            return bench_config(self.ws[0])
+        w = self.ws[-1]
+        return {"workload": self.name, "batch_per_gpu": self.batch, "tokens_per_request": w.n_tok[0],
+                "heads": w.heads, "layers": self.n_layers,
+                "caches": [{"name": c.name, "m": c.m[0], "layers": c.layers} for c in self.ws],
+                "kv_bytes_per_token": self.kv_bytes_per_token,
+                "l2": "flushed between timed steps (256 MB write, not timed)",
+                "timing": "CUDA graph replay of one step, CUDA events per step"}
+
+
+def run_gpu(args, rank: int, world: int, local_rank: int):
     import csa2_sparse_attention_decode_b200 as csa2
-    from csa2_sparse_attention_decode_b200.harness import DeviceWorkload
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    dw = DeviceWorkload(w, dev)
+    rn = Runner(args, dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
     k_scan = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     k_att = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    n_layers = len(w.layers)
+    n_layers = rn.n_layers
 
     # warm up eagerly once (first-call attribute set-up happens outside capture)
     with torch.cuda.stream(stream):
-        dw.restore(stream)
-        dw.step(stream)
+        rn.restore(stream)
+        rn.step(stream)
     stream.synchronize()
-    assert csa2.csa2_get_device_error(dw.cache, stream) == 0
+    for p in rn.parts:
+        assert csa2.csa2_get_device_error(p.cache, stream) == 0
 
     # torch only reports elapsed time between events it has recorded itself;
     # record each pair once so later records by the library are readable.
@@ -327,22 +393,22 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
     # One graph per layer: graph L brackets the attention of layer L (and the
     # index scan) with events, so the timed replays, taken in turn, measure
     # every layer's attention launch equally often.
-    scan_kernel = csa2.KERNEL_FLAT_SCORE if w.index == "flat" else csa2.KERNEL_BLOCK_SCORE
+    scan_kernel = csa2.KERNEL_FLAT_SCORE if rn.flat else csa2.KERNEL_BLOCK_SCORE
     csa2.csa2_set_profile_events(scan_kernel, *k_scan)
     graphs = []
     n0 = csa2.csa2_launch_count()
     for li in range(n_layers):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            dw.step(stream, attend_events=(li, k_att[0], k_att[1]))
+            rn.step(stream, attend_events=(li, k_att[0], k_att[1]))
         graphs.append(g)
     launches_per_step = (csa2.csa2_launch_count() - n0) / n_layers
     csa2.csa2_set_profile_events(scan_kernel, None, None)
 
     def one(i, timed_events=None):
         with torch.cuda.stream(stream):
-            if w.append:
-                dw.restore(stream)
+            if rn.append:
+                rn.restore(stream)
             flush.zero_()
             if timed_events:
                 timed_events[0].record(stream)
@@ -373,15 +439,13 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
     clocks = sampler.stop()
     max_total_ms = max_over_ranks(sum(step_ms), world, dev)
-    value = job_throughput(world, w.batch, args.steps, max_total_ms)
+    value = job_throughput(world, rn.batch, args.steps, max_total_ms)
 
     # ---- end to end: pinned host inputs -> device, replay, outputs -> host
-    ins = [x for li, mode in enumerate(w.layers) for x in
-           ((dw.layers[li][0],) + ((dw.layers[li][1], dw.layers[li][2]) if mode != "reuse" else ()))]
-    if w.append:
-        ins += list(dw.new)
+    ins = rn.inputs()
+    outs = rn.outs()
     host_in = [x.detach().cpu().pin_memory() for x in ins]
-    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in dw.outs]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
     h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = sum(x.numel() * x.element_size() for x in host_out)
     e2e_steps = max(3, min(args.steps, 200))
@@ -389,25 +453,25 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
     for i in range(e2e_steps + 3):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            if w.append:
-                dw.restore(stream)
+            if rn.append:
+                rn.restore(stream)
             flush.zero_()
             a.record(stream)
             for d, h in zip(ins, host_in):
                 d.copy_(h, non_blocking=True)
             graphs[i % n_layers].replay()
-            for h, o in zip(host_out, dw.outs):
+            for h, o in zip(host_out, outs):
                 h.copy_(o, non_blocking=True)
             b.record(stream)
         stream.synchronize()
         if i >= 3:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_value = job_throughput(world, w.batch, e2e_steps, max_over_ranks(sum(e2e_ms), world, dev))
+    e2e_value = job_throughput(world, rn.batch, e2e_steps, max_over_ranks(sum(e2e_ms), world, dev))
 
     # ---- roofline: attention (the largest share of the step's kernel time)
     # and the index scan, both timed live with CUDA events on the launching
     # stream over the timed region
-    ab = algorithmic_bytes(w)
+    ab = schedule_bytes(rn.ws)
     peak, peak_src = measured_peak_hbm()
     step_avg_ms = max_total_ms / args.steps
     att_avg_ms = statistics.mean(att_ms)
@@ -423,21 +487,25 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int, local_rank: int):
                 "step_frac": ab["step"] / (step_avg_ms / 1e3) / 1e9 / peak,
                 "step_algorithmic_bytes": ab["step"]}
     scan_avg_ms = statistics.mean(scan_ms)
-    scan_bytes = ab["block_summaries"] if w.index != "flat" else ab["index"]
+    # the events bracket the step's last scan: the last cache with a Full layer
+    scanned = [w for w in rn.ws if "full" in w.layers and w.index != "none"][-1]
+    last = algorithmic_bytes(scanned)
+    scan_bytes = (last["block_summaries"] if not rn.flat else last["index"]) / scanned.layers.count("full")
     scan_gbs = scan_bytes / (scan_avg_ms / 1e3) / 1e9
-    roofline_scan = {"bound": "hbm", "kernel": "score_umma_kernel (block-summary scan)" if w.index != "flat"
+    roofline_scan = {"bound": "hbm", "kernel": "score_umma_kernel (block-summary scan)" if not rn.flat
                      else "score_umma_kernel (flat key scan)", "achieved": scan_gbs, "peak": peak,
                      "peak_source": peak_src, "unit": "GB/s", "frac": scan_gbs / peak,
-                     "traffic": known_traffic("block_scan") if w.index != "flat" else None,
+                     "traffic": known_traffic("block_scan") if not rn.flat else None,
                      "kernel_ms": scan_avg_ms, "algorithmic_bytes_per_launch": scan_bytes}
 
     line = None
     if rank == 0:
-        cpu = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
+        cpu = (cpu_baseline(rn.ws[0]) if (world == 1 and not args.no_cpu_baseline and len(rn.ws) == 1)
+               else None)
         line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": step_avg_ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "fp8/bf16 MMA, fp32 accumulate", "data": "synthetic",
-                "config": bench_config(w),
+                "config": rn.config(),
                 "roofline": roofline, "roofline_index_scan": roofline_scan, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
@@ -454,7 +522,8 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
-    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--config", type=int, default=3,
+                    help="0-4: the single-cache workloads of synth.workload; 5: the 40-layer schedule")
     ap.add_argument("--small", action="store_true", help="small variant of the workload (testing only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -466,12 +535,16 @@ def main():
         if backend == "nccl":
             torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
-    w = synth.workload(args.config, small=args.small)
     try:
         if args.impl == "reference":
-            run_reference(args, w, rank, world)
+            if args.config == 5:
+                if rank == 0:
+                    print(json.dumps({"impl": "reference", "unavailable": "the oracle arm times the single-cache "
+                                      "workloads (configs 0-4); the 40-layer schedule has no CPU timing"}), flush=True)
+            else:
+                run_reference(args, synth.workload(args.config, small=args.small), rank, world)
         else:
-            run_gpu(args, w, rank, world, local_rank)
+            run_gpu(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -211,8 +211,6 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             tma_prefetch_map(m_chunk);
             tma_prefetch_map(m_tile);
         }
-        TileIter it;
-        it.init(s_rows, s_pre, p.c.batch, i0, i1);
         int issued = 0;
         bool stop = false;
         const int n_win = (n_items + PW - 1) / PW;
@@ -220,14 +218,20 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         // window w + 1 are issued before window w's copies and consumed after
         // them, so their latency hides behind the copies.
         int e_[8], b_[8], pg_[8];
-        auto meta = [&](int w) {                    // lane 0: tiles of window w
+        auto meta = [&](int w) {                    // lane i: tile i of window w
             const int wb = w & 1, nw = min(PW, n_items - w * PW);
-            if (lane == 0)
-                for (int i = 0; i < nw; ++i, it.next()) {
-                    win_b[wb][i] = it.b;
-                    win_r0[wb][i] = it.t * TILE;
-                    win_n[wb][i] = (min(TILE, it.rows - it.t * TILE) + chunk_rows - 1) / chunk_rows;
+            if (lane < nw) {
+                const long long g = i0 + (long long)w * PW + lane;
+                int lo = 0, hi = p.c.batch;         // the last request with s_pre[b] <= g owns tile g
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s_pre[mid] <= g) lo = mid; else hi = mid;
                 }
+                const int t = (int)(g - s_pre[lo]);
+                win_b[wb][lane] = lo;
+                win_r0[wb][lane] = t * TILE;
+                win_n[wb][lane] = (min(TILE, s_rows[lo] - t * TILE) + chunk_rows - 1) / chunk_rows;
+            }
             __syncwarp();
         };
         auto issue_loads = [&](int w) {             // non-blocking: loads in flight

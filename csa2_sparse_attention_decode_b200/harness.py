@@ -6,7 +6,9 @@ in the workload's schedule) through the C ABI.
 Layer schedule (0539edu.com/news/5732216 §3, layer modes): a "full" layer
 indexes and attends, "reuse" layers attend with their group's top-k and their
 own query, a "reindex" layer rescores the Full layer's pool with its own
-indexer query and opens a new group.
+indexer query and opens a new group, and a "swa" layer attends to its window
+alone.  ScheduleWorkload chains several caches' layer runs into one
+whole-model step.
 """
 from __future__ import annotations
 
@@ -40,7 +42,10 @@ class DeviceWorkload:
         B = w.batch
         self.pool = torch.full((B, POOL), -1, dtype=torch.int32, device=self.device)
         self.pool_len = torch.zeros(B, dtype=torch.int32, device=self.device)
-        self.topk = [torch.full((B, TOPK), -1, dtype=torch.int32, device=self.device) for _ in range(2)]
+        # one top-k buffer per group (each Full / Reindex layer opens one), and
+        # a last one that stays all -1 for SWA-only layers
+        n_groups = max(1, sum(1 for m in w.layers if m in ("full", "reindex")))
+        self.topk = [torch.full((B, TOPK), -1, dtype=torch.int32, device=self.device) for _ in range(n_groups + 1)]
         odt = torch.float32 if out_fp32 else torch.bfloat16
         self.outs = [torch.zeros(B, w.heads, 512, dtype=odt, device=self.device) for _ in w.layers]
         self.layer_topk: List[int] = []     # which topk buffer each layer attended with
@@ -77,25 +82,26 @@ class DeviceWorkload:
         if w.append:
             lat, key, gate, n_new = self.new
             csa2_append(c, lat, key, gate, n_new, stream)
-        grp = 0
+        grp = -1
         self.layer_topk = []
         for li, mode in enumerate(w.layers):
             q, q_idx, hw = self.layers[li]
             if mode == "full":
-                grp = 0
+                grp += 1
                 m = INDEX_FLAT if w.index == "flat" else INDEX_FULL
                 csa2_index(c, m, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws, stream)
             elif mode == "reindex":
-                grp = 1
+                grp += 1
                 csa2_index(c, INDEX_REINDEX, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws, stream)
-            self.layer_topk.append(grp)
+            buf = len(self.topk) - 1 if mode == "swa" else grp
+            self.layer_topk.append(buf)
             # A Reuse layer's indices were produced by its group's first layer,
             # not by the kernel right before it: its gather may start early.
             flags = ATTEND_INPUTS_SETTLED if mode == "reuse" else 0
             timed = attend_events is not None and attend_events[0] == li
             if timed:
                 csa2_set_profile_events(KERNEL_ATTEND, attend_events[1], attend_events[2])
-            csa2_attend(c, q, self.topk[grp], SOFTMAX_SCALE, self.outs[li], self.ws, stream, flags=flags)
+            csa2_attend(c, q, self.topk[buf], SOFTMAX_SCALE, self.outs[li], self.ws, stream, flags=flags)
             if timed:
                 csa2_set_profile_events(KERNEL_ATTEND, None, None)
 
@@ -128,3 +134,30 @@ class DeviceWorkload:
         codes = sv[SWA_CODES_OFF:SWA_CODES_OFF + 128 * 512].view(128, 512).cpu()
         scale = sv[SWA_SCALE_OFF:SWA_SCALE_OFF + 512].view(torch.float32).cpu()
         return codes, scale
+
+
+class ScheduleWorkload:
+    """The device side of a synth.Schedule: one DeviceWorkload per cache,
+    stepped in the schedule's layer order."""
+
+    def __init__(self, sched: synth.Schedule, device="cuda", out_fp32: bool = False):
+        self.sched = sched
+        self.parts = [DeviceWorkload(w, device, out_fp32=out_fp32) for w in sched.caches]
+
+    @property
+    def caches(self):
+        return [p.cache for p in self.parts]
+
+    def restore(self, stream=None):
+        for p in self.parts:
+            p.restore(stream)
+
+    def step(self, stream=None, attend_events=None):
+        """attend_events = (global layer index, ev_start, ev_stop)."""
+        base = 0
+        for p in self.parts:
+            ev = None
+            if attend_events is not None and base <= attend_events[0] < base + len(p.w.layers):
+                ev = (attend_events[0] - base, attend_events[1], attend_events[2])
+            p.step(stream, attend_events=ev)
+            base += len(p.w.layers)

@@ -70,10 +70,11 @@ class Workload:
     m: List[int]                     # 1 (decoder-style) or 2 (encoder-style)
     index: str                       # "flat" or "hier"
     layers: List[str]                # per layer: "full" | "reuse" | "reindex"
-    append: bool                     # each step first appends m new tokens
+    append: bool                     # each step first appends new tokens (m of them, or append_tokens)
     needles: int = 0
     outliers: bool = True
     shuffled_pages: bool = False
+    append_tokens: int = 0           # tokens appended per step when set (1 in the 40-layer schedule)
 
     @property
     def n_entries(self) -> List[int]:
@@ -81,7 +82,9 @@ class Workload:
 
     @property
     def n_new(self) -> List[int]:
-        return list(self.m) if self.append else [0] * self.batch
+        if not self.append:
+            return [0] * self.batch
+        return [self.append_tokens] * self.batch if self.append_tokens else list(self.m)
 
     def capacity_entries(self, b: int) -> int:
         return (self.n_tok[b] + self.n_new[b]) // self.m[b]
@@ -129,6 +132,51 @@ def workload(cid: int, small: bool = False) -> Workload:
         return Workload(f"ragged-paged-B{B}", 4, B, 64, n_tok, m, "hier", ["full"], True,
                         shuffled_pages=True)
     raise ValueError(cid)
+
+
+@dataclasses.dataclass
+class Schedule:
+    """A whole-model decode step: several caches, each with its contiguous
+    run of layers, executed in `caches` order (layer order of the model)."""
+    name: str
+    caches: List[Workload]
+
+    @property
+    def batch(self) -> int:
+        return self.caches[0].batch
+
+    @property
+    def n_layers(self) -> int:
+        return sum(len(c.layers) for c in self.caches)
+
+    def kv_bytes_per_token(self) -> float:
+        """Global-KV bytes per context token over the KV-producing caches:
+        an entry (288 B FP4 row + 128 B FP8 key) covers m tokens."""
+        return sum(416.0 / c.m[0] for c in self.caches if c.index != "none")
+
+
+def schedule40(small: bool = False) -> Schedule:
+    """The 40-layer CSA2 decode schedule (0539edu.com/news/5732216 §3 layer
+    modes; daiw.net million-token-cost: four layers produce global KV):
+      layers 0-1   SWA only, each over its own 128-token window;
+      layers 2-19  three encoder groups (m = 2) of Full + 5 Reuse, one cache each;
+      layers 20-39 decoder (m = 1), one cache: Full + 3 Reuse, then four
+                   groups of Reindex + 3 Reuse over the Full layer's pool.
+    Every cache holds T context tokens and appends one token per step (an
+    m = 2 cache completes an entry every other step).  Seeded like the other
+    workloads; cache c uses seed 10 + c."""
+    B, T = (2, 40000) if small else (4, 1 << 20)
+    tag = f"csa2-40-layer-B{B}-T{T}"
+    caches = []
+    for i in range(2):
+        caches.append(Workload(f"{tag}-swa{i}", 10 + i, B, 64, [min(T, SWA)] * B, [1] * B, "none", ["swa"], True,
+                               append_tokens=1))
+    for g in range(3):
+        caches.append(Workload(f"{tag}-enc{g}", 12 + g, B, 64, [T] * B, [2] * B, "hier", ["full"] + ["reuse"] * 5,
+                               True, append_tokens=1))
+    dec = ["full", "reuse", "reuse", "reuse"] + ["reindex", "reuse", "reuse", "reuse"] * 4
+    caches.append(Workload(f"{tag}-dec", 15, B, 64, [T] * B, [1] * B, "hier", dec, True, append_tokens=1))
+    return Schedule(tag, caches)
 
 
 # ---------------------------------------------------------------- draws

@@ -77,3 +77,55 @@ def check_attention(got: torch.Tensor, ref: np.ndarray, what=""):
     worst = np.unravel_index(np.argmax(err - tol), err.shape)
     assert (err <= tol).all(), f"{what}: max excess {float((err - tol)[worst]):.3g} at {worst}: got {g[worst]} ref {ref[worst]}"
     return float(err.max())
+
+
+def check_step(w, dw, refs, check_needles=False):
+    """Run one step of DeviceWorkload dw and check every stage of every
+    layer against the oracle (conditional on the GPU's block set)."""
+    import csa2_sparse_attention_decode_b200 as csa2
+    from csa2_sparse_attention_decode_b200.harness import SOFTMAX_SCALE
+
+    dw.step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    swaps = 0
+    for b in range(w.batch):
+        ref = refs[b]
+        pool = dw.pool[b].cpu().numpy()
+        plen = int(dw.pool_len[b])
+        group_topk = {}
+        for li, mode in enumerate(w.layers):
+            q, q_idx, hw = dw.layers[li]
+            qb, wb = bits(q_idx[b]), hw[b].cpu().numpy()
+            grp = dw.layer_topk[li]
+            gtop = dw.topk[grp][b].cpu().numpy()
+            if mode in ("full", "reindex"):
+                exact = {}
+
+                def score_of(e, qb=qb, wb=wb, exact=exact):
+                    if e not in exact:
+                        exact[e] = float(oracle.score_f64(qb, wb, ref.keys8[e:e + 1])[0])
+                    return exact[e]
+
+                if w.index == "flat":
+                    rtop = oracle.index_flat(qb, wb, ref.keys8)
+                else:
+                    if mode == "full":
+                        # blocks: the GPU pool's block set vs the oracle's block top-k
+                        gblocks = np.unique(pool[:plen] // 8)
+                        bs = oracle.score_f64(qb, wb, ref.summ)
+                        rblocks = oracle.topk(bs.astype(np.float32), 2048)
+                        swaps += check_swaps(gblocks, rblocks, lambda x: bs[x], f"req {b} blocks")
+                        rpool, rplen = oracle.expand_pool(gblocks.astype(np.int32), ref.n_entries)
+                        assert plen == rplen and np.array_equal(pool[:plen], rpool[:rplen]), b
+                    # conditional: the oracle's top-512 inside the GPU's pool
+                    rtop = oracle.index_pool(qb, wb, ref.keys8, pool, plen)
+                swaps += check_swaps(gtop, rtop, score_of, f"req {b} layer {li} top-k")
+                assert np.all(np.diff(gtop[gtop >= 0]) > 0) and (gtop[len(gtop[gtop >= 0]):] == -1).all()
+                if check_needles and mode == "full":
+                    needles = synth.needle_entries(w, b).numpy()
+                    assert set(needles.tolist()) <= set(gtop.tolist()), "needle missed"
+                group_topk[grp] = gtop
+            r = ref.attend(bits(q[b]), gtop, SOFTMAX_SCALE)
+            check_attention(dw.outs[li][b], r, f"req {b} layer {li}")
+    return swaps

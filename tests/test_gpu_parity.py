@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import OracleRequest, bits, check_attention, check_swaps
+from parity_util import OracleRequest, bits, check_attention, check_step, check_swaps
 
 pytestmark = pytest.mark.gpu
 
@@ -115,60 +115,13 @@ def test_append_matches_oracle(cid):
 
 
 # ------------------------------------------------------------------ index + attend, end to end
-def _check_step(w, dw, refs, check_needles=False):
-    dw.step()
-    torch.cuda.synchronize()
-    assert csa2.csa2_get_device_error(dw.cache) == 0
-    swaps = 0
-    for b in range(w.batch):
-        ref = refs[b]
-        pool = dw.pool[b].cpu().numpy()
-        plen = int(dw.pool_len[b])
-        group_topk = {}
-        for li, mode in enumerate(w.layers):
-            q, q_idx, hw = dw.layers[li]
-            qb, wb = bits(q_idx[b]), hw[b].cpu().numpy()
-            grp = dw.layer_topk[li]
-            gtop = dw.topk[grp][b].cpu().numpy()
-            if mode in ("full", "reindex"):
-                exact = {}
-
-                def score_of(e, qb=qb, wb=wb, exact=exact):
-                    if e not in exact:
-                        exact[e] = float(oracle.score_f64(qb, wb, ref.keys8[e:e + 1])[0])
-                    return exact[e]
-
-                if w.index == "flat":
-                    rtop = oracle.index_flat(qb, wb, ref.keys8)
-                else:
-                    if mode == "full":
-                        # blocks: the GPU pool's block set vs the oracle's block top-k
-                        gblocks = np.unique(pool[:plen] // 8)
-                        bs = oracle.score_f64(qb, wb, ref.summ)
-                        rblocks = oracle.topk(bs.astype(np.float32), 2048)
-                        swaps += check_swaps(gblocks, rblocks, lambda x: bs[x], f"req {b} blocks")
-                        rpool, rplen = oracle.expand_pool(gblocks.astype(np.int32), ref.n_entries)
-                        assert plen == rplen and np.array_equal(pool[:plen], rpool[:rplen]), b
-                    # conditional: the oracle's top-512 inside the GPU's pool
-                    rtop = oracle.index_pool(qb, wb, ref.keys8, pool, plen)
-                swaps += check_swaps(gtop, rtop, score_of, f"req {b} layer {li} top-k")
-                assert np.all(np.diff(gtop[gtop >= 0]) > 0) and (gtop[len(gtop[gtop >= 0]):] == -1).all()
-                if check_needles and mode == "full":
-                    needles = synth.needle_entries(w, b).numpy()
-                    assert set(needles.tolist()) <= set(gtop.tolist()), "needle missed"
-                group_topk[grp] = gtop
-            r = ref.attend(bits(q[b]), gtop, SOFTMAX_SCALE)
-            check_attention(dw.outs[li][b], r, f"req {b} layer {li}")
-    return swaps
-
-
 @pytest.mark.parametrize("cid", [0, 1, 2, 3, 4])
 @pytest.mark.parametrize("out_fp32", [True, False])
 def test_step_matches_oracle(cid, out_fp32):
     w = synth.workload(cid, small=True)
     dw = DeviceWorkload(w, out_fp32=out_fp32)
     refs = [OracleRequest(w, b, w.n_tok[b] + w.n_new[b]) for b in range(w.batch)]
-    _check_step(w, dw, refs, check_needles=(cid == 1))
+    check_step(w, dw, refs, check_needles=(cid == 1))
 
 
 def test_sharp_softmax_variant():
@@ -178,7 +131,7 @@ def test_sharp_softmax_variant():
     q, q_idx, hw = dw.layers[0]
     dw.layers[0] = ((q.float() * math.sqrt(512)).to(torch.bfloat16), q_idx, hw)
     refs = [OracleRequest(w, b, w.n_tok[b]) for b in range(w.batch)]
-    _check_step(w, dw, refs)
+    check_step(w, dw, refs)
 
 
 def _exact_index_check(w, dw, refs):
