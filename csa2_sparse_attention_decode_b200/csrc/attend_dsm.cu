@@ -372,27 +372,36 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
                 v[u][r] = (i < hi4 && tile_live[r]) ? reinterpret_cast<const float4 *>(cluster.map_shared_rank(Ob, r))[i]
                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        float4 acc[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            acc[u] = v[u][0];
+#pragma unroll
+            for (int r = 1; r < NTILES; ++r) {
+                acc[u].x += v[u][r].x; acc[u].y += v[u][r].y; acc[u].z += v[u][r].z; acc[u].w += v[u][r].w;
+            }
+        }
+        // Every remote read of this CTA has returned: tell the cluster, and
+        // wait for the others only after the output stores.
+        asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int i = lo4 + tid + u * THREADS;
             const int hh = i / (CSA2_LATENT / 4), d4 = i % (CSA2_LATENT / 4);
             if (i >= hi4 || hh >= nh) continue;
-            float4 acc = v[u][0];
-#pragma unroll
-            for (int r = 1; r < NTILES; ++r) {
-                acc.x += v[u][r].x; acc.y += v[u][r].y; acc.z += v[u][r].z; acc.w += v[u][r].w;
-            }
             const size_t o = ((size_t)b * heads + hg0 + hh) * CSA2_LATENT + 4 * d4;
             if (out_is_fp32) {
-                *reinterpret_cast<float4 *>((float *)out + o) = acc;
+                *reinterpret_cast<float4 *>((float *)out + o) = acc[u];
             } else {
-                __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+                __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y),
+                               hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
                 uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
                 *reinterpret_cast<uint2 *>((__nv_bfloat16 *)out + o) = pk;
             }
         }
     }
-    cluster.sync();                                       // no CTA leaves while its buffer is read
+    // No CTA leaves while another may still read its partials.
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
     fence_before_sync();
     __syncthreads();
     if (warp == 0) {

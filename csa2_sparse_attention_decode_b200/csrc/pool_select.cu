@@ -12,8 +12,8 @@
 // 128, at most 16384 / NC) and keeps the
 // order-preserving keys of its scores in shared memory; the cluster then runs
 // the selection of select.cuh over them and writes the selected pool ids.
-// Scoring roles (256 threads):
-//   warps 5-7   look up the page of every 8-row run of the CTA's rows, then
+// Scoring roles (384 threads):
+//   warps 5-11  look up the page of every 8-row run of the CTA's rows, then
 //               copy the runs (8 rows x 128 B of FP8 keys) with 16-byte
 //               asynchronous copies into an 8-stage ring of 128-row tiles,
 //               128-byte swizzled;
@@ -41,10 +41,10 @@ using namespace umma;
 
 namespace {
 
-constexpr int NT = 256;
+constexpr int NT = 384;
 constexpr int TILE = 128;
 constexpr int STAGES = 8;
-constexpr int NPROD = 96;                                // producer threads (warps 5-7)
+constexpr int NPROD = NT - 5 * 32;                       // producer threads (warps 5-11): more copies in flight
 constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;         // 16 KB
 // Shared-memory layout for NC CTAs per request (rows per CTA at most POOL/NC).
 template <int NC>
@@ -87,7 +87,7 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
 }
 
 __device__ __forceinline__ void bar_workers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ void bar_producers() { asm volatile("bar.sync 2, 96;" ::: "memory"); }
+__device__ __forceinline__ void bar_producers() { asm volatile("bar.sync 2, %0;" ::"n"(NPROD) : "memory"); }
 
 // 16-byte asynchronous global -> shared copy (L2 only), and an arrival on an
 // mbarrier once every copy this thread issued before it has landed (the
