@@ -252,3 +252,34 @@ def test_bad_page_id_sets_error():
     lat, key, gate = synth.tokens(w, 0, 0, 2048, "cuda")
     csa2.csa2_prefill(dw.cache, 0, 0, 2048, lat.contiguous(), key.contiguous(), gate.contiguous())
     assert csa2.csa2_get_device_error(dw.cache) == 1
+
+
+# ------------------------------------------------------------------ edge cases
+def test_empty_request_and_partial_head_group():
+    """A batch whose second request holds no tokens at all, with 40 heads (a
+    full 32-head group plus a partial one): the empty request gets an empty
+    top-k and a zero output; the other matches the oracle."""
+    w = synth.Workload("edge-B2-H40", 7, 2, 40, [3000, 0], [1, 1], "flat", ["full"], False, outliers=False)
+    dw = DeviceWorkload(w, out_fp32=True)
+    refs = [OracleRequest(w, 0, 3000)]
+    dw.step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    top = dw.topk[0].cpu().numpy()
+    assert (top[1] == -1).all()
+    assert torch.count_nonzero(dw.outs[0][1]) == 0
+    q, q_idx, hw = dw.layers[0]
+    rtop = oracle.index_flat(bits(q_idx[0]), hw[0].cpu().numpy(), refs[0].keys8)
+    assert np.array_equal(top[0], rtop)
+    r = refs[0].attend(bits(q[0]), top[0], SOFTMAX_SCALE)
+    check_attention(dw.outs[0][0], r, "request 0, 40 heads")
+
+
+def test_reindex_layer_over_short_pool():
+    """A request short enough that its pool is every entry (fewer than 2048
+    blocks): Full and Reindex both select from it exactly."""
+    w = synth.Workload("short-hier-B1", 8, 1, 64, [5000], [1], "hier", ["full", "reuse", "reindex", "reuse"], False)
+    dw = DeviceWorkload(w, out_fp32=True)
+    refs = [OracleRequest(w, 0, 5000)]
+    check_step(w, dw, refs)
+    assert int(dw.pool_len[0]) == 5000

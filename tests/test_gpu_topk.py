@@ -77,3 +77,10 @@ def test_topk_ragged_batch():
     r = _rng(11)
     rows = [r.standard_normal(int(n)).astype(np.float32) for n in (0, 5, 600, 16384, 40000, 2047, 2048, 2049)]
     _run(rows, 2048, stride=40000)
+
+
+def test_topk_rows_past_cluster_shared_memory():
+    # 600,000 keys: more per CTA than a 16-CTA cluster keeps in shared memory,
+    # so the selection re-reads the scores from global memory
+    r = _rng(600000)
+    _run([r.standard_normal(600000).astype(np.float32), np.round(r.standard_normal(600000) * 2) / 2], 2048)
