@@ -36,12 +36,12 @@ namespace {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace layout (all regions 256-byte aligned):
-//   scores_a [batch][row_stride] f32  row scores (entries or blocks)
-//   scores_b [batch][16384]      f32  pool scores
+//   scores   [batch][row_stride] f32  row scores of the block or flat scan
 //   blocks   [batch][2048]       i32  selected blocks (FULL)
-//   part_ml  [batch][10][heads][2] f32, part_o [batch][10][heads][512] f32
+// The pool's scores stay in shared memory (pool_select.cu) and attention
+// merges its splits inside a cluster (attend_dsm.cu): neither needs more.
 struct Workspace {
-    float *scores_a, *scores_b, *part_ml, *part_o;
+    float *scores;
     int32_t *blocks;
     int64_t row_stride;
     size_t bytes;
@@ -53,11 +53,9 @@ Workspace layout(void *base, int32_t batch, int32_t heads, int32_t max_entries)
     w.row_stride = ((int64_t)max_entries + 3) & ~(int64_t)3;
     size_t off = 0;
     auto take = [&](size_t n) { size_t o = off; off = align256(off + n); return (char *)base + o; };
-    w.scores_a = (float *)take(sizeof(float) * (size_t)batch * (size_t)w.row_stride);
-    w.scores_b = (float *)take(sizeof(float) * (size_t)batch * CSA2_POOL);
+    (void)heads;
+    w.scores = (float *)take(sizeof(float) * (size_t)batch * (size_t)w.row_stride);
     w.blocks = (int32_t *)take(sizeof(int32_t) * (size_t)batch * CSA2_MAX_BLOCKS);
-    w.part_ml = (float *)take(sizeof(float) * (size_t)batch * ATT_SPLITS * heads * 2);
-    w.part_o = (float *)take(sizeof(float) * (size_t)batch * ATT_SPLITS * heads * CSA2_LATENT);
     w.bytes = off;
     return w;
 }
@@ -132,17 +130,17 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaSuccess;
     if (mode == CSA2_INDEX_FLAT) {
-        e = launch_score(c, ROWS_KEYS, q_idx, w, nullptr, nullptr, W.scores_a, W.row_stride, max_entries, s);
+        e = launch_score(c, ROWS_KEYS, q_idx, w, nullptr, nullptr, W.scores, W.row_stride, max_entries, s);
         if (e == cudaSuccess)
-            e = launch_select(c, ROWS_KEYS, W.scores_a, W.row_stride, nullptr, nullptr, CSA2_TOPK, topk, CSA2_TOPK,
+            e = launch_select(c, ROWS_KEYS, W.scores, W.row_stride, nullptr, nullptr, CSA2_TOPK, topk, CSA2_TOPK,
                               0, nullptr, nullptr, max_entries, s);
         return from_cuda(e);
     }
     if (mode == CSA2_INDEX_FULL) {
         const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
-        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores_a, W.row_stride, max_blocks, s);
+        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores, W.row_stride, max_blocks, s);
         if (e == cudaSuccess)
-            e = launch_select(c, ROWS_SUMMARIES, W.scores_a, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS,
+            e = launch_select(c, ROWS_SUMMARIES, W.scores, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS,
                               W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, max_blocks, s);
         if (e != cudaSuccess) return from_cuda(e);
     }
@@ -174,8 +172,8 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
     Workspace W = layout(ws, cache->batch, heads, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
     if (flags & ~CSA2_ATTEND_INPUTS_SETTLED) return CSA2_ERR_INVALID_ARG;
-    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, flags, W.part_o,
-                                   W.part_ml, (cudaStream_t)stream));
+    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, flags, nullptr,
+                                   nullptr, (cudaStream_t)stream));
 }
 
 csa2_status csa2_get_device_error(const csa2_cache *cache, int32_t *code_out, csa2_stream_t stream)
