@@ -31,7 +31,9 @@ INDEX_FLAT, INDEX_FULL, INDEX_REINDEX = 0, 1, 2
 
 EXPORTS = ("csa2_page_bytes", "csa2_swa_bytes", "csa2_workspace_bytes", "csa2_prefill", "csa2_append",
            "csa2_index", "csa2_attend", "csa2_get_device_error", "csa2_status_string", "csa2_set_profile_events",
-           "csa2_launch_count", "csa2_attend_noalloc", "csa2_topk")
+           "csa2_launch_count", "csa2_attend_noalloc", "csa2_topk", "csa2_shard_blocks", "csa2_shard_pool",
+           "csa2_shard_rescore", "csa2_shard_topk", "csa2_attend_partial", "csa2_combine")
+MAX_SHARDS = 8
 ATTEND_NOALLOC_MAX_ROWS = 512
 KERNEL_BLOCK_SCORE, KERNEL_FLAT_SCORE, KERNEL_POOL_SCORE, KERNEL_SELECT, KERNEL_ATTEND, KERNEL_COMBINE = range(6)
 
@@ -72,6 +74,12 @@ def _load():
         "csa2_attend_noalloc": (C.c_int, [P, I32, P, P, C.c_float, P, I32, P]),
         "csa2_launch_count": (C.c_uint64, []),
         "csa2_topk": (C.c_int, [P, C.c_int64, P, I32, I32, P, P]),
+        "csa2_shard_blocks": (C.c_int, [P, P, P, P, P, P, P, SZ, P]),
+        "csa2_shard_pool": (C.c_int, [P, P, I32, P, P, P, P, P]),
+        "csa2_shard_rescore": (C.c_int, [P, P, P, P, P, P, P, P, P]),
+        "csa2_shard_topk": (C.c_int, [P, P, I32, P, P, P, P]),
+        "csa2_attend_partial": (C.c_int, [P, I32, P, P, C.c_float, I32, P, P, C.c_uint32, P]),
+        "csa2_combine": (C.c_int, [I32, P, P, I32, I32, P, I32, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -230,3 +238,65 @@ def csa2_attend_noalloc(cache: Cache, q, topk, scale: float, out, stream=None) -
     if st not in (0, 2):
         raise CSA2Error("csa2_attend_noalloc", st)
     return int(st)
+
+
+# ---------------------------------------------------------------- sequence shards
+def _ptrs(ts):
+    """Host array of the device pointers of tensors ts (kept alive by the caller)."""
+    if not 1 <= len(ts) <= MAX_SHARDS:
+        raise ValueError(f"1..{MAX_SHARDS} shards, got {len(ts)}")
+    arr = (C.c_void_p * len(ts))(*[_ptr(t).value for t in ts])
+    return C.cast(arr, C.c_void_p), arr
+
+
+def _bits16(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+
+
+def csa2_shard_blocks(cache, entry_offset, q_idx, w, block_ids, block_scores, ws, stream=None):
+    _check("csa2_shard_blocks", lib.csa2_shard_blocks(cache.ref, _ptr(entry_offset), _ptr(_bits16(q_idx)), _ptr(w),
+                                                      _ptr(block_ids), _ptr(block_scores), _ptr(ws), ws.numel(),
+                                                      _stream(stream)))
+
+
+def csa2_shard_pool(cache, entry_offset, cand_ids, cand_scores, pool, pool_len, stream=None):
+    pi, ki = _ptrs(cand_ids)
+    ps, ks = _ptrs(cand_scores)
+    _check("csa2_shard_pool", lib.csa2_shard_pool(cache.ref, _ptr(entry_offset), len(cand_ids), pi, ps, _ptr(pool),
+                                                  _ptr(pool_len), _stream(stream)))
+    del ki, ks
+
+
+def csa2_shard_rescore(cache, entry_offset, q_idx, w, pool, pool_len, ids, scores, stream=None):
+    _check("csa2_shard_rescore", lib.csa2_shard_rescore(cache.ref, _ptr(entry_offset), _ptr(_bits16(q_idx)), _ptr(w),
+                                                        _ptr(pool), _ptr(pool_len), _ptr(ids), _ptr(scores),
+                                                        _stream(stream)))
+
+
+def csa2_shard_topk(cache, entry_offset, cand_ids, cand_scores, topk, stream=None):
+    pi, ki = _ptrs(cand_ids)
+    ps, ks = _ptrs(cand_scores)
+    _check("csa2_shard_topk", lib.csa2_shard_topk(cache.ref, _ptr(entry_offset), len(cand_ids), pi, ps, _ptr(topk),
+                                                  _stream(stream)))
+    del ki, ks
+
+
+def csa2_attend_partial(cache, q, topk, scale: float, with_window: bool, o, lse, stream=None, flags: int = 0):
+    assert o.dtype == torch.float32 and lse.dtype == torch.float32
+    _check("csa2_attend_partial", lib.csa2_attend_partial(cache.ref, int(q.shape[1]), _ptr(_bits16(q)), _ptr(topk),
+                                                          float(scale), 1 if with_window else 0, _ptr(o), _ptr(lse),
+                                                          flags, _stream(stream)))
+
+
+def csa2_combine(o_parts, lse_parts, out, stream=None):
+    """out [batch, heads, 512] (bf16 or f32) = log-sum-exp merge of the
+    partial results o_parts[s] [batch, heads, 512] f32 with lse_parts[s]
+    [batch, heads] f32."""
+    if len(o_parts) != len(lse_parts):
+        raise ValueError("one lse per partial output")
+    po, ko = _ptrs(o_parts)
+    pl, kl = _ptrs(lse_parts)
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    _check("csa2_combine", lib.csa2_combine(len(o_parts), po, pl, int(out.shape[0]), int(out.shape[1]), _ptr(out),
+                                            fp32, _stream(stream)))
+    del ko, kl

@@ -25,6 +25,8 @@
 //      distributed shared memory; each live tile writes exp(m - M) / L times
 //      its partial O into its own shared memory; each CTA then sums one fifth
 //      of the output over the live tiles, reading their buffers remotely.
+// Partial mode (sequence-sharded decode): ATT_NO_WINDOW leaves the window
+// tile empty, and `lse` receives ln sum_j exp(scale * q.v_j) per head.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -114,7 +116,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
 
 __global__ void __cluster_dims__(NTILES, 1, 1) __launch_bounds__(THREADS, 1)
 attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads, const int32_t *topk, float scale,
-                  void *out, int out_is_fp32, uint32_t flags)
+                  void *out, int out_is_fp32, uint32_t flags, float *lse)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -141,7 +143,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     auto gather = [&]() {
         const int n_tok = c.n_tokens[b];
         const int n_entries = n_entries_of(c, b);
-        const int nv = max(0, min(n_tok, CSA2_SWA));
+        const int nv = (flags & ATT_NO_WINDOW) ? 0 : max(0, min(n_tok, CSA2_SWA));
         uint8_t *vrow = Vs + (2 * qtr) * V_SLAB + row * 128;
         const int sw = row & 7;
         if (tile < CSA2_TOPK / KT) {
@@ -341,6 +343,8 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         for (int r = 0; r < NTILES; ++r)
             if (mr[r] != -INFINITY) L += __expf(mr[r] - M) * cluster.map_shared_rank(&l_s[0], r)[tid];
         fac_s[tid] = (live && M != -INFINITY && L > 0.0f) ? __expf(m_s[tid] - M) / L : 0.0f;
+        if (lse && tile == 0 && tid < nh)
+            lse[(size_t)b * heads + hg0 + tid] = (M != -INFINITY && L > 0.0f) ? M + logf(L) : -INFINITY;
         if (tid < NTILES) tile_live[tid] = cluster.map_shared_rank(&m_s[0], tid)[0] != -INFINITY;
     }
     __syncthreads();
@@ -428,7 +432,7 @@ bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch)
 }  // namespace
 
 cudaError_t launch_attend_dsm(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                              void *out, int out_is_fp32, uint32_t flags, cudaStream_t st)
+                              void *out, int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse)
 {
     static bool attr_done[64] = {};
     int dev = 0;
@@ -444,7 +448,7 @@ cudaError_t launch_attend_dsm(const CacheView &c, int heads, const uint16_t *q, 
     dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);
     LaunchScope scope(CSA2_KERNEL_ATTEND, st);
     return launch_pdl(attend_dsm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, map_q, c, heads, topk, scale, out,
-                      out_is_fp32, flags);
+                      out_is_fp32, flags, lse);
 }
 
 }  // namespace csa2

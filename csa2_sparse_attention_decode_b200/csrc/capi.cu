@@ -176,6 +176,112 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
                                    nullptr, (cudaStream_t)stream));
 }
 
+// ------------------------------------------------------------ sequence shards
+csa2_status csa2_shard_blocks(const csa2_cache *shard, const int32_t *entry_offset, const uint16_t *q_idx,
+                              const float *w, int32_t *block_ids, float *block_scores, void *ws, size_t ws_bytes,
+                              csa2_stream_t stream)
+{
+    csa2_status st = check_cache(shard);
+    if (st != CSA2_OK) return st;
+    if (!entry_offset || !q_idx || !w || !block_ids || !block_scores || !ws || !aligned(ws, 256) ||
+        !aligned(q_idx, 16))
+        return CSA2_ERR_INVALID_ARG;
+    const int max_entries = shard->max_pages * CSA2_PAGE_ENTRIES;
+    Workspace W = layout(ws, shard->batch, 1, max_entries);
+    if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
+    CacheView c = make_view(shard);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
+    cudaError_t e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores, W.row_stride, max_blocks, s);
+    if (e == cudaSuccess)
+        e = launch_select(c, ROWS_SUMMARIES, W.scores, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS, block_ids,
+                          CSA2_MAX_BLOCKS, 0, nullptr, nullptr, max_blocks, s, block_scores, entry_offset, 3);
+    return from_cuda(e);
+}
+
+static_assert(MAX_SHARDS == CSA2_MAX_SHARDS, "one shard limit for the ABI and the kernels");
+
+namespace {
+csa2_status shard_lists(int32_t n_shards, const int32_t *const *ids, const float *const *scores, ShardLists &l)
+{
+    if (n_shards < 1 || n_shards > CSA2_MAX_SHARDS || !ids || !scores) return CSA2_ERR_INVALID_ARG;
+    l = ShardLists{};
+    for (int i = 0; i < n_shards; ++i) {
+        if (!ids[i] || !scores[i]) return CSA2_ERR_INVALID_ARG;
+        l.ids[i] = ids[i];
+        l.scores[i] = scores[i];
+    }
+    return CSA2_OK;
+}
+}  // namespace
+
+csa2_status csa2_shard_pool(const csa2_cache *shard, const int32_t *entry_offset, int32_t n_shards,
+                            const int32_t *const *cand_ids, const float *const *cand_scores, int32_t *pool,
+                            int32_t *pool_len, csa2_stream_t stream)
+{
+    csa2_status st = check_cache(shard);
+    if (st != CSA2_OK) return st;
+    ShardLists l;
+    if ((st = shard_lists(n_shards, cand_ids, cand_scores, l)) != CSA2_OK) return st;
+    if (!entry_offset || !pool || !pool_len) return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_shard_merge(make_view(shard), entry_offset, n_shards, l, 1, pool, pool_len,
+                                        (cudaStream_t)stream));
+}
+
+csa2_status csa2_shard_rescore(const csa2_cache *shard, const int32_t *entry_offset, const uint16_t *q_idx,
+                               const float *w, const int32_t *pool, const int32_t *pool_len, int32_t *ids,
+                               float *scores, csa2_stream_t stream)
+{
+    csa2_status st = check_cache(shard);
+    if (st != CSA2_OK) return st;
+    if (!entry_offset || !q_idx || !w || !pool || !pool_len || !ids || !scores || !aligned(q_idx, 16))
+        return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_pool_select(make_view(shard), q_idx, w, pool, pool_len, ids, (cudaStream_t)stream,
+                                        scores, entry_offset));
+}
+
+csa2_status csa2_shard_topk(const csa2_cache *shard, const int32_t *entry_offset, int32_t n_shards,
+                            const int32_t *const *cand_ids, const float *const *cand_scores, int32_t *topk,
+                            csa2_stream_t stream)
+{
+    csa2_status st = check_cache(shard);
+    if (st != CSA2_OK) return st;
+    ShardLists l;
+    if ((st = shard_lists(n_shards, cand_ids, cand_scores, l)) != CSA2_OK) return st;
+    if (!entry_offset || !topk) return CSA2_ERR_INVALID_ARG;
+    return from_cuda(launch_shard_merge(make_view(shard), entry_offset, n_shards, l, 0, topk, nullptr,
+                                        (cudaStream_t)stream));
+}
+
+csa2_status csa2_attend_partial(const csa2_cache *cache, int32_t heads, const uint16_t *q, const int32_t *topk,
+                                float scale, int32_t with_window, float *o, float *lse, uint32_t flags,
+                                csa2_stream_t stream)
+{
+    csa2_status st = check_cache(cache);
+    if (st != CSA2_OK) return st;
+    if (heads <= 0 || heads > 128 || !q || !topk || !o || !lse) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(o, 16) || !aligned(q, 16)) return CSA2_ERR_INVALID_ARG;
+    if (flags & ~CSA2_ATTEND_INPUTS_SETTLED) return CSA2_ERR_INVALID_ARG;
+    if (!with_window) flags |= ATT_NO_WINDOW;
+    return from_cuda(launch_attend_dsm(make_view(cache), heads, q, topk, scale, o, 1, flags, (cudaStream_t)stream,
+                                       lse));
+}
+
+csa2_status csa2_combine(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts, int32_t batch,
+                         int32_t heads, void *out, int32_t out_is_fp32, csa2_stream_t stream)
+{
+    if (n_parts < 1 || n_parts > CSA2_MAX_SHARDS || !o_parts || !lse_parts || !out) return CSA2_ERR_INVALID_ARG;
+    if (batch <= 0 || heads <= 0 || heads > 128 || (int64_t)batch * heads > 0x7fffffff || !aligned(out, 16))
+        return CSA2_ERR_INVALID_ARG;
+    PartList p{};
+    for (int i = 0; i < n_parts; ++i) {
+        if (!o_parts[i] || !lse_parts[i] || !aligned(o_parts[i], 16)) return CSA2_ERR_INVALID_ARG;
+        p.o[i] = o_parts[i];
+        p.lse[i] = lse_parts[i];
+    }
+    return from_cuda(launch_combine(n_parts, p, batch, heads, out, out_is_fp32, (cudaStream_t)stream));
+}
+
 csa2_status csa2_get_device_error(const csa2_cache *cache, int32_t *code_out, csa2_stream_t stream)
 {
     if (!cache || !cache->error || !code_out) return CSA2_ERR_INVALID_ARG;

@@ -30,12 +30,14 @@ constexpr size_t SEL_SMEM = (size_t)(SEL_CAP + 2 * sel::CAND + 2 * sel::RANK_MAX
 // element i is i, or ids[b][i] when ids != nullptr.  With expand the selected
 // ids are block numbers: the pool of their entries (< n_entries) is written
 // to pool[b][0..16384) in ascending order and its length to pool_len[b].
+// Optionally the selected scores go to vals[b][0..k) (-inf padded) and
+// (id_off[b] >> id_shift) is added to every written id.
 // CTA r owns the contiguous index range [r*chunk, (r+1)*chunk) and stages
 // its keys in shared memory (or re-reads global memory when chunk > SEL_CAP).
 template <int NC>
 __device__ __forceinline__ void select_body(CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,
                       const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
-                      int32_t *pool_len)
+                      int32_t *pool_len, float *vals, const int32_t *id_off, int id_shift)
 {
     extern __shared__ uint32_t dsm[];
     const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
@@ -102,13 +104,18 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     o.pool = pool;
     o.pool_len = pool_len;
     o.n_entries = n_entries;
+    o.vals = vals;
+    o.id_off = id_off;
+    o.id_shift = id_shift;
     sel::select_core<NC, SEL_THREADS>(bf, b, n, chunk, lo, cnt, k, kmin, kmax, o);
 }
 
 #define CSA2_SELECT_ARGS                                                                                      \
     CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,               \
-        const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool, int32_t *pool_len
-#define CSA2_SELECT_PASS c, src, scores, score_stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len
+        const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool, int32_t *pool_len,    \
+        float *vals, const int32_t *id_off, int id_shift
+#define CSA2_SELECT_PASS \
+    c, src, scores, score_stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift
 
 template <int NC>
 __global__ void __launch_bounds__(SEL_THREADS, 1) select_cluster_kernel(CSA2_SELECT_ARGS)
@@ -124,7 +131,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_cta_kernel(CSA2_SELECT_
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
-                          int32_t *pool_len, int max_n, cudaStream_t st)
+                          int32_t *pool_len, int max_n, cudaStream_t st, float *vals, const int32_t *id_off,
+                          int id_shift)
 {
     static bool attr_done[64] = {};
     static int cluster_size[64] = {};
@@ -151,12 +159,14 @@ cudaError_t launch_select(const CacheView &c, int src, const float *scores, int6
     LaunchScope scope(CSA2_KERNEL_SELECT, st);
     if (max_n <= SEL_CAP)   // fits one CTA's shared memory: no cluster barriers on the path
         return launch_pdl(select_cta_kernel, dim3(1, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores, stride,
-                          pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
+                          pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift);
     if (nc == 16)
         return launch_pdl_cluster(select_cluster_kernel<16>, dim3(16, c.batch), dim3(SEL_THREADS), smem, st, 16, c,
-                                  src, scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
+                                  src, scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len,
+                                  vals, id_off, id_shift);
     return launch_pdl_cluster(select_cluster_kernel<8>, dim3(8, c.batch), dim3(SEL_THREADS), smem, st, 8, c, src,
-                              scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len);
+                              scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals,
+                              id_off, id_shift);
 }
 
 }  // namespace csa2

@@ -9,11 +9,14 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
                          const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st);
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
-                          int32_t *pool_len, int max_n, cudaStream_t st);
+                          int32_t *pool_len, int max_n, cudaStream_t st, float *vals = nullptr,
+                          const int32_t *id_off = nullptr, int id_shift = 0);
 // Exact rescoring of the pool fused with its top-512 selection (one cluster
-// per request); writes the selected pool ids, ascending, -1 padded.
+// per request); writes the selected pool ids, ascending, -1 padded, and
+// optionally their scores (-inf padded) with id_off[b] added to every id.
 cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const float *w, const int32_t *pool,
-                               const int32_t *pool_len, int32_t *topk, cudaStream_t st);
+                               const int32_t *pool_len, int32_t *topk, cudaStream_t st, float *topk_scores = nullptr,
+                               const int32_t *id_off = nullptr);
 cudaError_t launch_prefill(const CacheView &c, int req, int m, int tok_begin, int n_tok, int n_tok_final,
                            const float *lat, const float *key, const float *gate, cudaStream_t st);
 cudaError_t launch_append(const CacheView &c, const float *lat, const float *key, const float *gate,
@@ -22,9 +25,28 @@ cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, cons
                           void *out, int out_is_fp32, uint32_t flags, float *part_o, float *part_ml, cudaStream_t st);
 
 // Attention with the split merge inside a cluster (distributed shared memory):
-// the csa2_attend path.  Needs no scratch.
+// the csa2_attend path.  Needs no scratch.  With lse != nullptr it also
+// writes ln sum_j exp(scale * q.v_j) per (request, head) ([batch][heads]).
 cudaError_t launch_attend_dsm(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                              void *out, int out_is_fp32, uint32_t flags, cudaStream_t st);
+                              void *out, int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse = nullptr);
+// Internal attention flag (beside CSA2_ATTEND_INPUTS_SETTLED): no window keys.
+constexpr uint32_t ATT_NO_WINDOW = 1u << 8;
+// Sequence-sharded decode (shard.cu): global top-k over the shards' lists,
+// keeping this shard's part.  expand = 1: block lists -> pool; 0: entry
+// lists -> topk.
+constexpr int MAX_SHARDS = 8;
+struct ShardLists {
+    const int32_t *ids[MAX_SHARDS];
+    const float *scores[MAX_SHARDS];
+};
+cudaError_t launch_shard_merge(const CacheView &c, const int32_t *entry_offset, int n_shards, const ShardLists &l,
+                               int expand, int32_t *out, int32_t *pool_len, cudaStream_t st);
+struct PartList {
+    const float *o[MAX_SHARDS];
+    const float *lse[MAX_SHARDS];
+};
+cudaError_t launch_combine(int n_parts, const PartList &p, int batch, int heads, void *out, int out_is_fp32,
+                           cudaStream_t st);
 // Attention with the scaled split partials exchanged through global scratch
 // `part_o` ([batch][5][heads][512] fp32): the csa2_attend_noalloc path.
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,

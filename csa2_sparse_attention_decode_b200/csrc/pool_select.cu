@@ -103,7 +103,7 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
 
 template <int NC>
 __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const uint16_t *q_idx, const float *w, const int32_t *pool, const int32_t *pool_len,
-                   int32_t *topk)
+                   int32_t *topk, float *topk_scores, const int32_t *id_off)
 {
     using Lay = Layout<NC>;
     constexpr int RUNS = Lay::RUNS;
@@ -297,6 +297,9 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     o.pool = nullptr;
     o.pool_len = nullptr;
     o.n_entries = n_entries;
+    o.vals = topk_scores;
+    o.id_off = id_off;
+    o.id_shift = 0;
     sel::select_core<NC, NT>(bf, b, n, chunk, lo, cnt, CSA2_TOPK, kmin, kmax, o);
 
     fence_before_sync();
@@ -310,7 +313,8 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
 }  // namespace
 
 cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const float *w, const int32_t *pool,
-                               const int32_t *pool_len, int32_t *topk, cudaStream_t st)
+                               const int32_t *pool_len, int32_t *topk, cudaStream_t st, float *topk_scores,
+                               const int32_t *id_off)
 {
     // 16 CTAs per request where the device can schedule such clusters
     // (shorter per-CTA row ranges), else 8.
@@ -338,9 +342,9 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
     LaunchScope scope(CSA2_KERNEL_POOL_SCORE, st);
     if (nc == 16)
         return launch_pdl_cluster(pool_select_kernel<16>, dim3(16, c.batch), dim3(NT), Layout<16>::SMEM_BYTES, st, 16,
-                                  c, q_idx, w, pool, pool_len, topk);
+                                  c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
     return launch_pdl_cluster(pool_select_kernel<8>, dim3(8, c.batch), dim3(NT), Layout<8>::SMEM_BYTES, st, 8, c,
-                              q_idx, w, pool, pool_len, topk);
+                              q_idx, w, pool, pool_len, topk, topk_scores, id_off);
 }
 
 }  // namespace csa2

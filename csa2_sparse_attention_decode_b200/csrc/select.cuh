@@ -62,7 +62,16 @@ struct Out {
     int expand;                  // ids are block numbers: write their entries to pool
     int32_t *pool, *pool_len;
     int n_entries;               // entries of the request (expand mode)
+    float *vals;                 // optional: the selected scores beside out (-inf padded)
+    const int32_t *id_off;       // optional: (id_off[b] >> id_shift) is added to every written id
+    int id_shift;
 };
+
+// Inverse of ord_key (a -0 score comes back as +0).
+__device__ __forceinline__ float key_score(uint32_t key)
+{
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
 
 // Inclusive scan over threads 0..255 (warps 0..7); every thread of the CTA
 // must call it.  Returns the prefix for threads < 256.
@@ -328,7 +337,9 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
                 o.pool[(size_t)b * CSA2_POOL + pos * CSA2_BLOCK + j] = en < o.n_entries ? en : -1;
             }
         } else {
-            o.out[(size_t)b * o.out_stride + pos] = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
+            const int id = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
+            o.out[(size_t)b * o.out_stride + pos] = (o.id_off && id >= 0) ? id + (o.id_off[b] >> o.id_shift) : id;
+            if (o.vals) o.vals[(size_t)b * o.out_stride + pos] = key_score(key_at(gi - lo));
         }
     };
     auto pad_tail = [&]() {
@@ -337,14 +348,18 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
                 for (int i = kk * CSA2_BLOCK + tid; i < CSA2_POOL; i += NT) o.pool[(size_t)b * CSA2_POOL + i] = -1;
                 if (n == 0 && tid == 0) o.pool_len[b] = 0;
             } else {
-                for (int i = kk + tid; i < k; i += NT) o.out[(size_t)b * o.out_stride + i] = -1;
+                for (int i = kk + tid; i < k; i += NT) {
+                    o.out[(size_t)b * o.out_stride + i] = -1;
+                    if (o.vals) o.vals[(size_t)b * o.out_stride + i] = -INFINITY;
+                }
             }
         }
     };
-    if ((ranked || take_all) && bf.keys) {
+    if ((ranked || take_all) && bf.keys && !o.vals) {
         // Every decision is local: one pass compacts each warp's chosen
         // elements in place (over keys it has already read), then the
-        // warps' and CTAs' counts place them.
+        // warps' and CTAs' counts place them.  (Not with scores out: the
+        // compaction overwrites the keys.)
         uint32_t c = 0;
         for (int it = 0; it < seg; it += 32) {
             const int e = wid * seg + it + lane;

@@ -227,6 +227,95 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
  * is read after the previous kernel completes. */
 #define CSA2_ATTEND_INPUTS_SETTLED 1u
 
+/* Sequence-sharded decode of long requests --------------------------------
+ * The pages describe decode on one device; they do not split a request.
+ * These calls split each request's entries over G shards (normally one per
+ * GPU), so that G devices share one long request's block scan, pool
+ * rescoring and gathers, and they reproduce the unsharded result: the
+ * selections are exactly those of csa2_index FULL / REINDEX (the global top-k
+ * of a union of per-shard top-k lists equals the top-k of the whole, under
+ * the same order: score descending, ties to the lower global index), and the
+ * attention equals csa2_attend's up to fp32 rounding of the final merge.
+ *
+ * Shards.  Shard s of request b holds the request's global entries
+ * [entry_offset[b], entry_offset[b] + N_s) in a csa2_cache of its own (its
+ * n_tokens / m = N_s; its page table lists only its pages).  entry_offset is
+ * a device int32 array [batch], a multiple of 8 (of 64 to keep pages whole);
+ * a bad offset sets CSA2_DEV_BAD_REQUEST and the request selects nothing.
+ * Shards are numbered in increasing offset and cover the request without
+ * gaps.  Only the LAST shard holds the SWA window and takes appends; its
+ * n_tokens must count at least min(total tokens, 128) tokens so that its
+ * window is the request's.  Exchanged lists are passed as host arrays of
+ * n_shards device pointers, in shard order, each to a [batch][k] array (the
+ * buffers of an all-gather, or peers' memory mapped into this process); at
+ * most CSA2_MAX_SHARDS shards.
+ *
+ * One Full layer on shard s:
+ *   1. csa2_shard_blocks    local top-2048 blocks by summary score
+ *   2. exchange             every shard's block ids + scores to every shard
+ *   3. csa2_shard_pool      global top-2048 blocks; this shard's ones -> its pool
+ *   4. csa2_shard_rescore   exact pool rescoring, local top-512
+ *   5. exchange             every shard's top-512 ids + scores
+ *   6. csa2_shard_topk      global top-512; this shard's entries -> its topk
+ *   7. csa2_attend_partial  attention over its topk (+ window on the last
+ *                           shard): normalised output and log-sum-exp
+ *   8. exchange             outputs and log-sum-exps
+ *   9. csa2_combine         log-sum-exp merge of the shards' outputs
+ * A Reindex layer runs steps 4-9 on the Full layer's shard pool; a Reuse
+ * layer runs steps 7-9 with its group's shard topk.                        */
+#define CSA2_MAX_SHARDS 8
+
+/* Step 1.  The top min(2048, ceil(N_s/8)) blocks of this shard by summary
+ * score (as csa2_index FULL scores them): block_ids [batch][2048] gets
+ * GLOBAL block numbers (local + entry_offset/8) ascending, -1 padded;
+ * block_scores [batch][2048] their f32 scores, -inf padded.  ws: workspace
+ * of csa2_workspace_bytes() for this shard's cache. */
+csa2_status csa2_shard_blocks(const csa2_cache *shard, const int32_t *entry_offset,
+                              const uint16_t *q_idx, const float *w,
+                              int32_t *block_ids, float *block_scores,
+                              void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/* Step 3.  Over the n_shards lists of step 1 (cand_ids[s] / cand_scores[s],
+ * each [batch][2048]): the global top-2048 blocks; those inside this shard
+ * are expanded, ascending, into its pool [batch][16384] as LOCAL entry
+ * indices (entries past N_s become -1), pool_len [batch] counts them. */
+csa2_status csa2_shard_pool(const csa2_cache *shard, const int32_t *entry_offset, int32_t n_shards,
+                            const int32_t *const *cand_ids, const float *const *cand_scores,
+                            int32_t *pool, int32_t *pool_len, csa2_stream_t stream);
+
+/* Step 4.  Exact rescoring of this shard's pool (csa2_index REINDEX's
+ * arithmetic) and its top min(512, pool_len): ids [batch][512] get GLOBAL
+ * entry indices ascending, -1 padded; scores [batch][512] f32, -inf padded. */
+csa2_status csa2_shard_rescore(const csa2_cache *shard, const int32_t *entry_offset,
+                               const uint16_t *q_idx, const float *w,
+                               const int32_t *pool, const int32_t *pool_len,
+                               int32_t *ids, float *scores, csa2_stream_t stream);
+
+/* Step 6.  Over the n_shards lists of step 4 (each [batch][512]): the global
+ * top-512 entries; those inside this shard go to topk [batch][512] as LOCAL
+ * entry indices, ascending, -1 padded. */
+csa2_status csa2_shard_topk(const csa2_cache *shard, const int32_t *entry_offset, int32_t n_shards,
+                            const int32_t *const *cand_ids, const float *const *cand_scores,
+                            int32_t *topk, csa2_stream_t stream);
+
+/* Step 7.  csa2_attend over the valid topk entries, plus the window only
+ * when with_window != 0, returning the pieces a merge needs:
+ * o [batch][heads][512] f32, normalised over this call's keys (zero without
+ * keys), and lse [batch][heads] f32 = ln sum_j exp(scale * q_h . v_j)
+ * (-inf without keys).  flags as csa2_attend.  No workspace. */
+csa2_status csa2_attend_partial(const csa2_cache *cache, int32_t heads, const uint16_t *q,
+                                const int32_t *topk, float scale, int32_t with_window,
+                                float *o, float *lse, uint32_t flags, csa2_stream_t stream);
+
+/* Step 9.  out[b][h] = sum_s exp(lse_s - L) o_s[b][h] with
+ * L = ln sum_s exp(lse_s) over the n_parts (1..CSA2_MAX_SHARDS) partial
+ * results o_parts[s] [batch][heads][512] f32 and lse_parts[s]
+ * [batch][heads] f32 (host arrays of device pointers); zero where every
+ * lse is -inf.  out is bf16 (out_is_fp32 = 0) or f32 (= 1). */
+csa2_status csa2_combine(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts,
+                         int32_t batch, int32_t heads, void *out, int32_t out_is_fp32,
+                         csa2_stream_t stream);
+
 /* Attention without a workspace ------------------------------------------
  * The pages have no counterpart to this call; it exists for callers that
  * cannot allocate device memory -- for instance code embedded in a host
@@ -262,7 +351,7 @@ typedef enum {
     CSA2_KERNEL_POOL_SCORE = 2,    /* FULL / REINDEX: exact pool rescoring     */
     CSA2_KERNEL_SELECT = 3,        /* radix top-k                              */
     CSA2_KERNEL_ATTEND = 4,        /* split-KV attention partials              */
-    CSA2_KERNEL_COMBINE = 5,       /* reserved: the merge runs inside ATTEND   */
+    CSA2_KERNEL_COMBINE = 5,       /* shard merges and csa2_combine            */
     CSA2_KERNEL_COUNT = 6
 } csa2_kernel_id;
 

@@ -73,6 +73,8 @@ def lib():
                 ("orc_index_pool", C.c_int, [P, P, P, P, C.c_int, P]),
                 ("orc_index_full", C.c_int, [P, P, P, P, C.c_int, P, P, P]),
                 ("orc_attend", None, [C.c_int, P, C.c_int, P, P, C.c_int, P, P, C.c_double, P]),
+                ("orc_attend_lse", None, [C.c_int, P, C.c_int, P, P, C.c_int, P, P, C.c_double, P, P]),
+                ("orc_lse_combine", None, [C.c_int, C.c_int, P, P, P]),
             ]:
                 f = getattr(L, name)
                 f.restype = res
@@ -284,4 +286,32 @@ def attend(q_bits, codes_sel, scales_sel, swa_codes, swa_scale, scale: float) ->
     out = np.empty((H, LATENT), np.float64)
     lib().orc_attend(H, _p(q_bits), codes_sel.shape[0], _p(codes_sel), _p(scales_sel),
                      swa_codes.shape[0], _p(swa_codes), _p(swa_scale), float(scale), _p(out))
+    return out
+
+
+def attend_lse(q_bits, codes_sel, scales_sel, swa_codes, swa_scale, scale: float):
+    """attend() plus, per head, ln sum_j exp(scale * q_h . v_j) (-inf when
+    there are no keys).  Returns (fp64 [H, 512], fp64 [H])."""
+    q_bits = _c(q_bits, np.uint16)
+    H = q_bits.shape[0]
+    codes_sel = _c(codes_sel, np.uint8).reshape(-1, CODE_BYTES)
+    scales_sel = _c(scales_sel, np.uint8).reshape(-1, SCALE_BYTES)
+    swa_codes = _c(swa_codes, np.uint8).reshape(-1, LATENT)
+    swa_scale = _c(swa_scale, np.float32).reshape(-1)
+    out = np.empty((H, LATENT), np.float64)
+    lse = np.empty(H, np.float64)
+    lib().orc_attend_lse(H, _p(q_bits), codes_sel.shape[0], _p(codes_sel), _p(scales_sel),
+                         swa_codes.shape[0], _p(swa_codes), _p(swa_scale), float(scale), _p(out), _p(lse))
+    return out, lse
+
+
+def lse_combine(o_parts, lse_parts) -> np.ndarray:
+    """Merge of attention results over disjoint key sets: o_parts [P, rows,
+    512], lse_parts [P, rows] -> [rows, 512] fp64."""
+    o_parts = _c(o_parts, np.float64)
+    lse_parts = _c(lse_parts, np.float64)
+    P, rows = lse_parts.shape
+    assert o_parts.shape == (P, rows, LATENT)
+    out = np.empty((rows, LATENT), np.float64)
+    lib().orc_lse_combine(P, rows, _p(o_parts), _p(lse_parts), _p(out))
     return out

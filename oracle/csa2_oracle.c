@@ -392,10 +392,12 @@ int orc_index_full(const uint16_t *q, const float *w, const uint8_t *keys8, cons
  * ====================================================================== */
 
 /* o_h = sum_j softmax_j(scale * q_h . v_j) v_j over n_sel FP4 rows and n_swa
- * FP8 rows.  q is bf16 [H][512]; out is fp64 [H][512]. */
-void orc_attend(int H, const uint16_t *q, int n_sel, const uint8_t *codes, const uint8_t *scales,
-                int n_swa, const uint8_t *swa_codes, const float *swa_scale, double scale,
-                double *out)
+ * FP8 rows.  q is bf16 [H][512]; out is fp64 [H][512].  When lse is not
+ * NULL it receives, per head, the log of the softmax denominator measured
+ * from zero: ln sum_j exp(scale * q_h . v_j) (-inf for an empty key set). */
+void orc_attend_lse(int H, const uint16_t *q, int n_sel, const uint8_t *codes, const uint8_t *scales,
+                    int n_swa, const uint8_t *swa_codes, const float *swa_scale, double scale,
+                    double *out, double *lse)
 {
     int n = n_sel + n_swa;
     double *v = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * OR_LATENT);
@@ -410,6 +412,7 @@ void orc_attend(int H, const uint16_t *q, int n_sel, const uint8_t *codes, const
     for (int h = 0; h < H; ++h) {
         double *o = out + (size_t)h * OR_LATENT;
         for (int d = 0; d < OR_LATENT; ++d) o[d] = 0.0;
+        if (lse) lse[h] = -INFINITY;
         if (n == 0) continue;
         double qd[OR_LATENT];
         for (int d = 0; d < OR_LATENT; ++d) qd[d] = orc_bf16_to_float(q[h * OR_LATENT + d]);
@@ -422,6 +425,7 @@ void orc_attend(int H, const uint16_t *q, int n_sel, const uint8_t *codes, const
         }
         double l = 0.0;
         for (int j = 0; j < n; ++j) { p[j] = exp(p[j] - mx); l += p[j]; }
+        if (lse) lse[h] = mx + log(l);
         for (int j = 0; j < n; ++j) {
             double pj = p[j] / l;
             for (int d = 0; d < OR_LATENT; ++d) o[d] += pj * v[(size_t)j * OR_LATENT + d];
@@ -429,6 +433,39 @@ void orc_attend(int H, const uint16_t *q, int n_sel, const uint8_t *codes, const
     }
     free(v);
     free(p);
+}
+
+void orc_attend(int H, const uint16_t *q, int n_sel, const uint8_t *codes, const uint8_t *scales,
+                int n_swa, const uint8_t *swa_codes, const float *swa_scale, double scale,
+                double *out)
+{
+    orc_attend_lse(H, q, n_sel, codes, scales, n_swa, swa_codes, swa_scale, scale, out, NULL);
+}
+
+/* Merge of attention results over disjoint parts of one key set: part s
+ * holds o_s (normalised over its keys) and lse_s = ln of its softmax
+ * denominator.  The whole set's denominator is sum_s exp(lse_s), so
+ *   o = sum_s exp(lse_s - L) o_s,   L = ln sum_s exp(lse_s),
+ * evaluated with the largest lse_s factored out.  Parts with lse_s = -inf
+ * (no keys) weigh nothing; with no keys at all the output is zero.
+ * o_parts [P][rows][512], lse_parts [P][rows], out [rows][512], fp64. */
+void orc_lse_combine(int n_parts, int rows, const double *o_parts, const double *lse_parts, double *out)
+{
+    for (int r = 0; r < rows; ++r) {
+        double mx = -INFINITY;
+        for (int s = 0; s < n_parts; ++s)
+            if (lse_parts[(size_t)s * rows + r] > mx) mx = lse_parts[(size_t)s * rows + r];
+        double *o = out + (size_t)r * OR_LATENT;
+        for (int d = 0; d < OR_LATENT; ++d) o[d] = 0.0;
+        if (mx == -INFINITY) continue;
+        double den = 0.0;
+        for (int s = 0; s < n_parts; ++s) den += exp(lse_parts[(size_t)s * rows + r] - mx);
+        for (int s = 0; s < n_parts; ++s) {
+            const double ws = exp(lse_parts[(size_t)s * rows + r] - mx) / den;
+            const double *os = o_parts + ((size_t)s * rows + r) * OR_LATENT;
+            for (int d = 0; d < OR_LATENT; ++d) o[d] += ws * os[d];
+        }
+    }
 }
 
 /* ======================================================================

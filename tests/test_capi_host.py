@@ -88,3 +88,36 @@ def test_invalid_arguments_rejected_before_launch(csa2):
     assert L.csa2_topk(good, 0, good, 4, 512, good, None) == 1
     assert L.csa2_get_device_error(None, None, None) == 1
     assert csa2.status_string(1) == "invalid argument"
+
+
+def test_sharded_calls_reject_invalid_arguments_before_launch(csa2):
+    L = csa2.lib
+    P = C.c_void_p
+    good = P(256 * 100)
+    c = _fake_cache(csa2)
+    lists = (C.c_void_p * 9)(*([256 * 200] * 9))
+    lp = C.cast(lists, C.c_void_p)
+    holes = (C.c_void_p * 2)(256 * 200, None)
+    hp = C.cast(holes, C.c_void_p)
+    # shard counts outside 1..8, a null list entry, null outputs
+    for n in (0, 9):
+        assert L.csa2_shard_pool(C.byref(c), good, n, lp, lp, good, good, None) == 1, n
+        assert L.csa2_shard_topk(C.byref(c), good, n, lp, lp, good, None) == 1, n
+        assert L.csa2_combine(n, lp, lp, 2, 64, good, 0, None) == 1, n
+    assert L.csa2_shard_pool(C.byref(c), good, 2, hp, lp, good, good, None) == 1
+    assert L.csa2_shard_topk(C.byref(c), good, 2, lp, hp, good, None) == 1
+    assert L.csa2_shard_pool(C.byref(c), None, 2, lp, lp, good, good, None) == 1
+    assert L.csa2_shard_topk(C.byref(c), good, 2, lp, lp, None, None) == 1
+    assert L.csa2_shard_blocks(C.byref(c), good, good, good, good, good, good, 16, None) == 1   # workspace
+    assert L.csa2_shard_blocks(C.byref(c), None, good, good, good, good, good, 1 << 30, None) == 1
+    assert L.csa2_shard_rescore(C.byref(c), good, good, good, good, good, good, None, None) == 1
+    assert L.csa2_shard_rescore(None, good, good, good, good, good, good, good, None) == 1
+    # partial attention: heads, null lse, unknown flag
+    assert L.csa2_attend_partial(C.byref(c), 0, good, good, 0.1, 1, good, good, 0, None) == 1
+    assert L.csa2_attend_partial(C.byref(c), 64, good, good, 0.1, 1, good, None, 0, None) == 1
+    assert L.csa2_attend_partial(C.byref(c), 64, good, good, 0.1, 1, good, good, 2, None) == 1
+    # combine: batch, heads, misaligned part
+    mis = (C.c_void_p * 2)(256 * 200, 256 * 200 + 4)
+    assert L.csa2_combine(2, lp, lp, 0, 64, good, 0, None) == 1
+    assert L.csa2_combine(2, lp, lp, 2, 129, good, 0, None) == 1
+    assert L.csa2_combine(2, C.cast(mis, C.c_void_p), lp, 2, 64, good, 0, None) == 1

@@ -353,3 +353,64 @@ def test_attention_closed_forms():
     swc, sws = oracle.swa_quant(lat[:3])
     o = oracle.attend(q, codes[:0], scales[:0], swc, sws, 0.0)
     assert np.allclose(o, np.broadcast_to((oracle.e4m3_decode(swc) * sws[:, None]).mean(0), o.shape), atol=1e-12)
+
+
+# ------------------------------------------------------------------ split attention: log-sum-exp and merge
+def _packed_rows(rng, n, spread=2.0):
+    lat = (rng.standard_normal((n, 512)) * spread).astype(np.float32)
+    packed = [oracle.pack_latent(r) for r in lat]
+    codes = np.stack([c for c, _ in packed]) if n else np.zeros((0, 256), np.uint8)
+    scales = np.stack([s for _, s in packed]) if n else np.zeros((0, 32), np.uint8)
+    return codes, scales
+
+
+def test_attention_lse_matches_torch_logsumexp_and_closed_forms():
+    rng = np.random.default_rng(21)
+    codes, scales = _packed_rows(rng, 30)
+    swa_c, swa_s = oracle.swa_quant((rng.standard_normal((6, 512)) * 30).astype(np.float32))
+    qb = bf16_bits(rng.standard_normal((8, 512)))
+    scale = 0.07
+    o, lse = oracle.attend_lse(qb, codes, scales, swa_c, swa_s, scale)
+    assert np.array_equal(o, oracle.attend(qb, codes, scales, swa_c, swa_s, scale))
+    v = np.concatenate([np.stack([oracle.unpack_latent(c, s) for c, s in zip(codes, scales)]),
+                        oracle.e4m3_decode(swa_c) * swa_s[:, None].astype(np.float64)])
+    logits = scale * (torch.from_numpy(oracle.bf16_bits_to_f64(qb)) @ torch.from_numpy(v).T)
+    assert np.allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=1e-13, atol=1e-13)
+    none_c, none_s = np.zeros((0, 512), np.uint8), np.zeros(0, np.float32)
+    # one key: lse = its logit
+    _, l1 = oracle.attend_lse(qb, codes[:1], scales[:1], none_c, none_s, scale)
+    assert np.allclose(l1, scale * (oracle.bf16_bits_to_f64(qb) @ v[0]), rtol=1e-13, atol=1e-13)
+    # q = 0 over n keys: every logit is 0, lse = ln n
+    _, l0 = oracle.attend_lse(np.zeros((3, 512), np.uint16), codes, scales, swa_c, swa_s, scale)
+    assert np.allclose(l0, math.log(36), rtol=0, atol=1e-13)
+    # no keys: -inf and a zero output
+    oe, le = oracle.attend_lse(qb, codes[:0], scales[:0], none_c, none_s, scale)
+    assert np.all(le == -np.inf) and not oe.any()
+
+
+def test_lse_combine_of_a_key_split_is_the_whole_attention():
+    rng = np.random.default_rng(22)
+    codes, scales = _packed_rows(rng, 50, spread=3.0)
+    swa_c, swa_s = oracle.swa_quant((rng.standard_normal((7, 512)) * 10).astype(np.float32))
+    qb = bf16_bits(rng.standard_normal((5, 512)) * 3)        # sharp logits
+    scale = 1 / math.sqrt(512)
+    none_c, none_s = np.zeros((0, 512), np.uint8), np.zeros(0, np.float32)
+    whole = oracle.attend(qb, codes, scales, swa_c, swa_s, scale)
+    # four parts: two slices of the FP4 rows, an empty part, the window alone
+    parts = [(codes[:17], scales[:17], none_c, none_s), (codes[17:], scales[17:], none_c, none_s),
+             (codes[:0], scales[:0], none_c, none_s), (codes[:0], scales[:0], swa_c, swa_s)]
+    res = [oracle.attend_lse(qb, c, s, wc, ws, scale) for c, s, wc, ws in parts]
+    o_parts = np.stack([r[0] for r in res])
+    l_parts = np.stack([r[1] for r in res])
+    merged = oracle.lse_combine(o_parts, l_parts)
+    assert np.allclose(merged, whole, rtol=1e-12, atol=1e-12)
+    # the order of the parts does not matter
+    perm = [3, 0, 2, 1]
+    assert np.allclose(oracle.lse_combine(o_parts[perm], l_parts[perm]), whole, rtol=1e-12, atol=1e-12)
+    # one part: the identity
+    assert np.allclose(oracle.lse_combine(o_parts[:1], l_parts[:1]), o_parts[0], rtol=0, atol=1e-15)
+    # every part empty: zero
+    z = oracle.lse_combine(np.zeros((2, 5, 512)), np.full((2, 5), -np.inf))
+    assert not z.any()
+    # a dropped weight (plain mean of the parts) is detectably wrong
+    assert not np.allclose(o_parts[[0, 1, 3]].mean(0), whole, atol=1e-6)
