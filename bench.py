@@ -105,8 +105,8 @@ def schedule_bytes(ws) -> dict:
 KNOWN_TRAFFIC = {
     "block_scan": {"bytes": 67_501_056 + 827_136, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
                    "sha256": "a3c2814836873bcbe6f19a489395cf2958005ce57066d43c01b840ceb548bc67"},
-    "attend": {"bytes": 1_556_736, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
-               "sha256": "ac956989221a0da834f71bd8fecd2b43d4efdf71429c3343dca7e3c5f91ff9ec"},
+    "attend": {"bytes": 1_558_528, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
+               "sha256": "8254d6e87582f7d08672457e44cb8c872e41906be0e79c0a122c9ea2475d5bc7"},
 }
 
 
@@ -330,12 +330,24 @@ class Runner:
             dw = DeviceWorkload(w, dev)
             self.name, self.ws, self.parts, self.step = w.name, [w], [dw], dw.step
             self.kv_bytes_per_token = None
+        self.sharded = None
+        if args.shards > 1:
+            # the sequence-sharded step, all shards on this one device
+            from csa2_sparse_attention_decode_b200.sharded import LocalShards
+            if args.config == 5 or w.index != "hier":
+                raise SystemExit("--shards runs the hierarchical single-cache workloads (configs 2-4)")
+            self.sharded = LocalShards(dw, args.shards)
+            self.step = self.sharded.step
+            self.name = f"{w.name}-seq-sharded-{args.shards}-on-1-GPU"
         self.batch = self.ws[0].batch
         self.n_layers = sum(len(w.layers) for w in self.ws)
         self.append = any(w.append for w in self.ws)
         self.flat = any(w.index == "flat" for w in self.ws)
 
     def restore(self, stream):
+        if self.sharded is not None:
+            self.sharded.restore(stream)
+            return
         for p in self.parts:
             p.restore(stream)
 
@@ -353,6 +365,8 @@ class Runner:
         return ins
 
     def outs(self):
+        if self.sharded is not None:
+            return list(self.sharded.outs)
         return [o for p in self.parts for o in p.outs]
 
     def pack_io(self, dev):
@@ -390,9 +404,18 @@ class Runner:
                 p.layers[li] = (q, q_idx, hw)
             if p.w.append:
                 p.new = tuple(next(vin) for _ in p.new)
-            p.outs = [next(vout) for _ in p.outs]
+            if self.sharded is None:
+                p.outs = [next(vout) for _ in p.outs]
+        if self.sharded is not None:
+            self.sharded.outs = [next(vout) for _ in self.sharded.outs]
 
     def config(self) -> dict:
+        if self.sharded is not None:
+            c = bench_config(self.ws[0])
+            c.update(workload=self.name, shards=self.sharded.n_shards,
+                     shard_entry_offsets=self.sharded.offsets,
+                     shards_run="one after another on this one GPU; exchanges are pointer lists")
+            return c
         if len(self.ws) == 1:
             return bench_config(self.ws[0])
         w = self.ws[-1]
@@ -402,6 +425,48 @@ class Runner:
                 "kv_bytes_per_token": self.kv_bytes_per_token,
                 "l2": "flushed between timed steps (256 MB write, not timed)",
                 "timing": "CUDA graph replay of one step, CUDA events per step"}
+
+
+def sharded_attend_bytes(rn) -> float:
+    """Algorithmic bytes of the last shard's partial attention launches,
+    averaged over the step's layers: its selected FP4 rows, the window, q in,
+    the fp32 output and log-sum-exp out, and the top-k ids."""
+    from csa2_sparse_attention_decode_b200.sharded import _schedule
+    w, last = rn.ws[0], rn.sharded.shards[-1]
+    n_tok = last.cache.n_tokens.cpu().tolist()
+    total = 0.0
+    for li, mode, grp in _schedule(w.layers):
+        sel = (last.topk[grp] >= 0).sum(dim=1).cpu().tolist()
+        for b in range(w.batch):
+            total += (sel[b] * 288 + min(n_tok[b], 128) * 516 + w.heads * 512 * (2 + 4) + w.heads * 4
+                      + 512 * 4)
+    return total / len(w.layers)
+
+
+def per_shard_ms(rn, stream, flush, args) -> list:
+    """Device time of each shard's own work alone, per step (graph replays
+    with an L2 flush between them)."""
+    out = []
+    for s in range(rn.sharded.n_shards):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            rn.sharded.step(stream, only=s)
+        reps = max(3, min(args.steps, 200))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for i in range(reps + 3):
+                if rn.append:
+                    rn.restore(stream)
+                flush.zero_()
+                if i >= 3:
+                    evs[i - 3][0].record(stream)
+                g.replay()
+                if i >= 3:
+                    evs[i - 3][1].record(stream)
+        stream.synchronize()
+        out.append(statistics.mean(a.elapsed_time(b) for a, b in evs))
+        del g
+    return out
 
 
 def run_gpu(args, rank: int, world: int, local_rank: int):
@@ -537,7 +602,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     peak, peak_src = measured_peak_hbm()
     step_avg_ms = max_total_ms / args.steps
     att_avg_ms = statistics.mean(att_ms)
-    att_bytes = ab["attend"] / n_layers
+    att_bytes = ab["attend"] / n_layers if rn.sharded is None else sharded_attend_bytes(rn)
     att_gbs = att_bytes / (att_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": "attend_dsm_kernel", "achieved": att_gbs, "peak": peak,
                 "peak_source": peak_src, "unit": "GB/s", "frac": att_gbs / peak,
@@ -553,6 +618,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     scanned = [w for w in rn.ws if "full" in w.layers and w.index != "none"][-1]
     last = algorithmic_bytes(scanned)
     scan_bytes = (last["block_summaries"] if not rn.flat else last["index"]) / scanned.layers.count("full")
+    if rn.sharded is not None:   # the events bracket the last shard's scan
+        sc = rn.sharded.shards[-1].cache
+        scan_bytes = sum(-(-(int(t) // m) // 8) * 128 for t, m in zip(sc.n_tokens.cpu().tolist(), sc.m_host))
     scan_gbs = scan_bytes / (scan_avg_ms / 1e3) / 1e9
     roofline_scan = {"bound": "hbm", "kernel": "score_umma_kernel (block-summary scan)" if not rn.flat
                      else "score_umma_kernel (flat key scan)", "achieved": scan_gbs, "peak": peak,
@@ -560,10 +628,12 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                      "traffic": known_traffic("block_scan") if not rn.flat else None,
                      "kernel_ms": scan_avg_ms, "algorithmic_bytes_per_launch": scan_bytes}
 
+    per_shard = per_shard_ms(rn, stream, flush, args) if rn.sharded is not None else None
+
     line = None
     if rank == 0:
-        cpu = (cpu_baseline(rn.ws[0]) if (world == 1 and not args.no_cpu_baseline and len(rn.ws) == 1)
-               else None)
+        cpu = (cpu_baseline(rn.ws[0]) if (world == 1 and not args.no_cpu_baseline and len(rn.ws) == 1
+                                          and rn.sharded is None) else None)
         line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": step_avg_ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "fp8/bf16 MMA, fp32 accumulate", "data": "synthetic",
@@ -575,6 +645,13 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                                 "streams, overlapping the previous and next steps' compute"},
                 "gpu_launches": int(launches_per_step * args.steps),
                 "clocks": clocks}
+        if per_shard is not None:
+            # what each GPU of a G-GPU run would compute (its own shard's
+            # kernels and the merges), without the exchanges between GPUs
+            line["per_shard_ms_per_step"] = per_shard
+            roofline["kernel"] = "attend_dsm_kernel (the last shard's partial attention)"
+            roofline_scan["kernel"] = "score_umma_kernel (the last shard's block-summary scan)"
+            roofline["traffic"] = roofline_scan["traffic"] = None
         print(json.dumps(line), flush=True)
     del graphs
     return line
@@ -590,6 +667,8 @@ def main():
                     help="0-4: the single-cache workloads of synth.workload; 5: the 40-layer schedule")
     ap.add_argument("--small", action="store_true", help="small variant of the workload (testing only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shards", type=int, default=1,
+                    help="run the sequence-sharded step with this many shards, all on one GPU (configs 2-4)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -21,10 +21,11 @@
 //      product keeps ~16 bits of P), stored K-major as [head][key].
 //   5. O^T[512 x 32] = V^T . (P_hi + P_lo)^T        (4 dim chunks x 2 x 8
 //      MMAs; the V tile is read again as an MN-major operand)
-//   6. merge: the tiles exchange the per-head max m and sum l over
-//      distributed shared memory; each live tile writes exp(m - M) / L times
-//      its partial O into its own shared memory; each CTA then sums one fifth
-//      of the output over the live tiles, reading their buffers remotely.
+//   6. merge: each live tile writes its partial O into its own shared
+//      memory beside its per-head max m and sum l; after one cluster barrier
+//      each CTA reads every tile's (m, l), forms the weights exp(m - M) / L
+//      and sums one fifth of the output over the live tiles, reading their
+//      buffers remotely.
 // Partial mode (sequence-sharded decode): ATT_NO_WINDOW leaves the window
 // tile empty, and `lse` receives ln sum_j exp(scale * q.v_j) per head.
 #include <cuda_bf16.h>
@@ -125,7 +126,8 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     float *Ob = reinterpret_cast<float *>(Vs);
     __shared__ __align__(8) uint64_t bar_q, bar_s, bar_o;
     __shared__ uint32_t tmem_base;
-    __shared__ float m_s[HG], l_s[HG], fac_s[HG], red_m[KC][HG], red_l[KC][HG];
+    __shared__ float m_s[HG], l_s[HG], red_m[KC][HG], red_l[KC][HG];
+    __shared__ float mt_s[NTILES][HG], lt_s[NTILES][HG], fac_s[NTILES][HG];   // every tile's (m, l), weights
     __shared__ int tile_live[NTILES];
     cg::cluster_group cluster = cg::this_cluster();
 
@@ -329,28 +331,12 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
             l_s[tid] = 0.0f;
         }
     }
-    // ---- 6. merge the five tiles of this (request, head group)
-    cluster.sync();
-    if (tid < HG) {
-        float mr[NTILES], M = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < NTILES; ++r) {
-            mr[r] = cluster.map_shared_rank(&m_s[0], r)[tid];
-            M = fmaxf(M, mr[r]);
-        }
-        float L = 0.0f;
-#pragma unroll
-        for (int r = 0; r < NTILES; ++r)
-            if (mr[r] != -INFINITY) L += __expf(mr[r] - M) * cluster.map_shared_rank(&l_s[0], r)[tid];
-        fac_s[tid] = (live && M != -INFINITY && L > 0.0f) ? __expf(m_s[tid] - M) / L : 0.0f;
-        if (lse && tile == 0 && tid < nh)
-            lse[(size_t)b * heads + hg0 + tid] = (M != -INFINITY && L > 0.0f) ? M + logf(L) : -INFINITY;
-        if (tid < NTILES) tile_live[tid] = cluster.map_shared_rank(&m_s[0], tid)[0] != -INFINITY;
-    }
-    __syncthreads();
+    // ---- 6. merge the five tiles of this (request, head group).  Each live
+    // tile leaves its unscaled partial O^T as [head][dim] fp32 in its V
+    // region (free once the second product has completed) beside its
+    // per-head (m, l); after one cluster barrier every CTA forms all five
+    // tiles' weights exp(m_r - M) / L and sums its fifth of the output.
     if (live) {
-        // The second product has completed: the V tile is free for the
-        // scaled partial, [head][dim] fp32.
         wait_bar(&bar_o, 0, c.error);
         fence_after_sync();
         uint32_t rr[32];
@@ -358,9 +344,31 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         tmem_ld_wait();
         const int d = 128 * (warp >> 2) + 32 * (warp & 3) + lane;
 #pragma unroll
-        for (int j = 0; j < HG; ++j) Ob[j * CSA2_LATENT + d] = __uint_as_float(rr[j]) * fac_s[j];
+        for (int j = 0; j < HG; ++j) Ob[j * CSA2_LATENT + d] = __uint_as_float(rr[j]);
     }
-    cluster.sync();                                       // partials visible cluster-wide
+    cluster.sync();                                       // (m, l) and partials visible cluster-wide
+    if (tid < NTILES * HG) {
+        const int r = tid / HG, hh = tid % HG;
+        mt_s[r][hh] = cluster.map_shared_rank(&m_s[0], r)[hh];
+        lt_s[r][hh] = cluster.map_shared_rank(&l_s[0], r)[hh];
+    }
+    __syncthreads();
+    if (tid < HG) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < NTILES; ++r) M = fmaxf(M, mt_s[r][tid]);
+        float L = 0.0f;
+#pragma unroll
+        for (int r = 0; r < NTILES; ++r)
+            if (mt_s[r][tid] != -INFINITY) L += __expf(mt_s[r][tid] - M) * lt_s[r][tid];
+        const bool any = M != -INFINITY && L > 0.0f;
+#pragma unroll
+        for (int r = 0; r < NTILES; ++r)
+            fac_s[r][tid] = (any && mt_s[r][tid] != -INFINITY) ? __expf(mt_s[r][tid] - M) / L : 0.0f;
+        if (lse && tile == 0 && tid < nh) lse[(size_t)b * heads + hg0 + tid] = any ? M + logf(L) : -INFINITY;
+        if (tid < NTILES) tile_live[tid] = mt_s[tid][0] != -INFINITY;
+    }
+    __syncthreads();
     {
         // This CTA's fifth (at most 820 float4, two per thread): every remote
         // load of both is issued before any sum.
@@ -379,10 +387,15 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         float4 acc[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            acc[u] = v[u][0];
+            const int hh = min((lo4 + tid + u * THREADS) / (CSA2_LATENT / 4), HG - 1);
+            acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int r = 1; r < NTILES; ++r) {
-                acc[u].x += v[u][r].x; acc[u].y += v[u][r].y; acc[u].z += v[u][r].z; acc[u].w += v[u][r].w;
+            for (int r = 0; r < NTILES; ++r) {
+                const float f = fac_s[r][hh];
+                acc[u].x = fmaf(f, v[u][r].x, acc[u].x);
+                acc[u].y = fmaf(f, v[u][r].y, acc[u].y);
+                acc[u].z = fmaf(f, v[u][r].z, acc[u].z);
+                acc[u].w = fmaf(f, v[u][r].w, acc[u].w);
             }
         }
         // Every remote read of this CTA has returned: tell the cluster, and

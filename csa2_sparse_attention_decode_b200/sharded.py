@@ -30,9 +30,9 @@ from typing import List, Sequence
 
 import torch
 
-from . import (ATTEND_INPUTS_SETTLED, MAX_BLOCKS, PAGE_ENTRIES, POOL, SWA, TOPK, Cache, csa2_append,
-               csa2_attend_partial, csa2_cache, csa2_combine, csa2_shard_blocks, csa2_shard_pool, csa2_shard_rescore,
-               csa2_shard_topk, workspace)
+from . import (ATTEND_INPUTS_SETTLED, KERNEL_ATTEND, MAX_BLOCKS, PAGE_ENTRIES, POOL, SWA, TOPK, Cache, csa2_append,
+               csa2_attend_partial, csa2_cache, csa2_combine, csa2_set_profile_events, csa2_shard_blocks,
+               csa2_shard_pool, csa2_shard_rescore, csa2_shard_topk, workspace)
 
 # Shard boundaries are multiples of 128 entries: whole pages (64 entries),
 # whole blocks (8), and (times m) whole turns of the 128-slot window ring,
@@ -184,24 +184,38 @@ class LocalShards:
             self.shards[-1].cache.n_tokens.copy_(self.saved[0])
             self.shards[-1].cache.pending.copy_(self.saved[1])
 
-    def step(self, stream=None):
+    def step(self, stream=None, attend_events=None, only=None):
+        """One sharded decode step.  attend_events = (layer, ev_start,
+        ev_stop) brackets the last shard's attention of that layer.  only = s
+        runs shard s's own work alone (what one GPU of G would run, minus the
+        exchanges), reading the other shards' lists as the last full step
+        left them."""
         w, sh = self.dw.w, self.shards
-        if w.append:
+        mine = [x for i, x in enumerate(sh) if only is None or i == only]
+        if w.append and (only is None or only == len(sh) - 1):
             lat, key, gate, n_new = self.dw.new
             csa2_append(sh[-1].cache, lat, key, gate, n_new, stream)
         for li, mode, grp in _schedule(w.layers):
             q, q_idx, hw = self.dw.layers[li]
             if mode == "full":
-                lists = [s.blocks(q_idx, hw, stream) for s in sh]
-                for s in sh:
-                    s.pool_from([x[0] for x in lists], [x[1] for x in lists], stream)
+                for s in mine:
+                    s.blocks(q_idx, hw, stream)
+                for s in mine:
+                    s.pool_from([x.blk_ids for x in sh], [x.blk_scores for x in sh], stream)
             if mode in ("full", "reindex"):
-                lists = [s.rescore(q_idx, hw, stream) for s in sh]
-                for s in sh:
-                    s.topk_from(grp, [x[0] for x in lists], [x[1] for x in lists], stream)
+                for s in mine:
+                    s.rescore(q_idx, hw, stream)
+                for s in mine:
+                    s.topk_from(grp, [x.cand_ids for x in sh], [x.cand_scores for x in sh], stream)
             flags = ATTEND_INPUTS_SETTLED if mode == "reuse" else 0
-            parts = [s.attend(grp, q, self.scale, flags, stream) for s in sh]
-            sh[0].combine([p[0] for p in parts], [p[1] for p in parts], self.outs[li], stream)
+            timed = attend_events is not None and attend_events[0] == li
+            for s in mine:
+                if timed and s is mine[-1]:
+                    csa2_set_profile_events(KERNEL_ATTEND, attend_events[1], attend_events[2])
+                s.attend(grp, q, self.scale, flags, stream)
+                if timed and s is mine[-1]:
+                    csa2_set_profile_events(KERNEL_ATTEND, None, None)
+            sh[0].combine([x.o for x in sh], [x.lse for x in sh], self.outs[li], stream)
 
 
 class DistShard:
