@@ -105,8 +105,8 @@ def schedule_bytes(ws) -> dict:
 KNOWN_TRAFFIC = {
     "block_scan": {"bytes": 67_501_056 + 827_136, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
                    "sha256": "a3c2814836873bcbe6f19a489395cf2958005ce57066d43c01b840ceb548bc67"},
-    "attend": {"bytes": 1_558_528, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
-               "sha256": "8254d6e87582f7d08672457e44cb8c872e41906be0e79c0a122c9ea2475d5bc7"},
+    "attend": {"bytes": 1_560_320, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
+               "sha256": "9762f6cad1bf18be7ff484493bb488419c4bf06dabdd0bfe27644974904f3adf"},
 }
 
 
