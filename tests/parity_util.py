@@ -129,3 +129,26 @@ def check_step(w, dw, refs, check_needles=False):
             r = ref.attend(bits(q[b]), gtop, SOFTMAX_SCALE)
             check_attention(dw.outs[li][b], r, f"req {b} layer {li}")
     return swaps
+
+
+def sharded_topk(ls, grp, b) -> np.ndarray:
+    """Global top-k of group grp, request b, of a sharded.LocalShards step:
+    every shard's local ids (checked ascending, -1 padded) at its offset."""
+    ids = []
+    for s, sh in enumerate(ls.shards):
+        t = sh.topk[grp][b].cpu().numpy()
+        v = t[t >= 0]
+        assert np.all(np.diff(v) > 0) and (t[v.size:] == -1).all()
+        ids += (v + ls.offsets[s][b]).tolist()
+    return np.asarray(ids, np.int64)
+
+
+def sharded_pool(ls, b) -> np.ndarray:
+    """Global pool of request b of a sharded.LocalShards step."""
+    out = []
+    for s, sh in enumerate(ls.shards):
+        n = int(sh.pool_len[b])
+        p = sh.pool[b].cpu().numpy()
+        assert (p[:n] >= 0).all()
+        out += (p[:n] + ls.offsets[s][b]).tolist()
+    return np.asarray(out, np.int64)

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import bits, check_attention, check_swaps
+from parity_util import bits, check_attention, check_swaps, sharded_pool, sharded_topk
 
 pytestmark = pytest.mark.gpu
 
@@ -134,3 +134,36 @@ def test_fullsize_ragged_paged_64():
     order = np.argsort(w.n_tok)
     picks = sorted({int(order[0]), int(order[-1]), 3, 40})          # shortest, longest, an m=2 and an m=1 request
     _run(4, picks, n_entry_samples=128)
+
+
+@pytest.mark.parametrize("n_shards", [2, 4])
+def test_fullsize_reuse_group_1m_sharded(n_shards):
+    """The sequence-sharded step at full size, as bench.py --shards runs it:
+    for every request and layer the selections equal the unsharded step's
+    exactly; a sampled request's outputs against the oracle."""
+    from csa2_sparse_attention_decode_b200.sharded import LocalShards, _schedule
+    w = synth.workload(3)
+    dw = DeviceWorkload(w)
+    ls = LocalShards(dw, n_shards)
+    dw.step()
+    torch.cuda.synchronize()
+    un_top = [t.cpu().numpy().copy() for t in dw.topk]
+    un_pool, un_plen = dw.pool.cpu().numpy().copy(), dw.pool_len.cpu().numpy().copy()
+    un_layer = list(dw.layer_topk)
+    dw.restore()
+    ls.step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0
+    for b in range(w.batch):
+        assert np.array_equal(sharded_pool(ls, b), un_pool[b][: un_plen[b]]), b
+        for li, mode, grp in _schedule(w.layers):
+            u = un_top[un_layer[li]][b]
+            assert np.array_equal(sharded_topk(ls, grp, b), u[u >= 0]), (b, li)
+    b = 2
+    ref = SampledRequest(w, b, w.n_tok[b])
+    for li, mode, grp in _schedule(w.layers):
+        q = dw.layers[li][0][b]
+        ids = sharded_topk(ls, grp, b)
+        codes_s, scales_s, _ = ref.packed(ids)
+        r = oracle.attend(bits(q), codes_s, scales_s, ref.win[0], ref.win[1], SOFTMAX_SCALE)
+        check_attention(ls.outs[li][b], r, f"{w.name} sharded x{n_shards} req {b} layer {li}")

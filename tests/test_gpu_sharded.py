@@ -16,29 +16,9 @@ import torch
 
 import oracle
 import synth
-from parity_util import OracleRequest, bits, check_attention, check_swaps
+from parity_util import OracleRequest, bits, check_attention, check_swaps, sharded_pool, sharded_topk
 
 pytestmark = pytest.mark.gpu
-
-
-def _global_topk(ls, grp, b):
-    ids = []
-    for s, sh in enumerate(ls.shards):
-        t = sh.topk[grp][b].cpu().numpy()
-        v = t[t >= 0]
-        assert np.all(np.diff(v) > 0) and (t[v.size:] == -1).all()
-        ids += (v + ls.offsets[s][b]).tolist()
-    return np.asarray(ids, np.int64)
-
-
-def _global_pool(ls, b):
-    out = []
-    for s, sh in enumerate(ls.shards):
-        n = int(sh.pool_len[b])
-        p = sh.pool[b].cpu().numpy()
-        assert (p[:n] >= 0).all()
-        out += (p[:n] + ls.offsets[s][b]).tolist()
-    return np.asarray(out, np.int64)
 
 
 def _run_and_check(w, n_shards, out_fp32=True):
@@ -65,11 +45,11 @@ def _run_and_check(w, n_shards, out_fp32=True):
         for li, mode, grp in _schedule(w.layers):
             q, q_idx, hw = dw.layers[li]
             qb, wb = bits(q_idx[b]), hw[b].cpu().numpy()
-            gtop = _global_topk(ls, grp, b)
+            gtop = sharded_topk(ls, grp, b)
             u = un_top[un_layer[li]][b]
             assert np.array_equal(gtop, u[u >= 0]), f"req {b} layer {li}: sharded top-k differs from unsharded"
             if mode == "full":
-                gpool = _global_pool(ls, b)
+                gpool = sharded_pool(ls, b)
                 assert np.array_equal(gpool, un_pool[b][: un_plen[b]]), f"req {b}: pool differs from unsharded"
                 gblocks = np.unique(gpool // 8)
                 bs = oracle.score_f64(qb, wb, ref.summ)
