@@ -8,18 +8,18 @@
 // 0539edu.com/news/5732216 §3 (fp4_e2m1 global KV with an e4m3 scale per 16
 // channels; fp8 SWA with a 128-token window).
 //
-// Grid (5 tiles, ceil(heads / 32) head groups, batch); the five tiles of one
+// Grid (5 tiles, ceil(heads / 16) head groups, batch); the five tiles of one
 // (request, head group) form a cluster.  Tiles 0-3 are the top-512 entries,
 // tile 4 the SWA window.  512 threads: while gathering, thread t owns key row
 // t & 127 and a quarter (t >> 7) of its 512 channels.
-//   1. q (bf16, 32 heads x 512) -> smem by TMA, K-major, 128-byte swizzle.
+//   1. q (bf16, 16 heads x 512) -> smem by TMA, K-major, 128-byte swizzle.
 //   2. gather + dequantise 128 keys to bf16 (exact: e2m1 x e4m3 and
 //      e4m3 x 2^e all fit bf16) -> smem V tile, K-major, swizzled.
-//   3. S^T[128 keys x 32 heads] = V . Q^T            (32 MMAs, fp32 in TMEM)
+//   3. S^T[128 keys x 16 heads] = V . Q^T            (32 MMAs, fp32 in TMEM)
 //   4. softmax per head over the tile's keys through a smem transpose;
 //      P = exp(scale*S - m) is split into bf16 hi + lo parts (the second
 //      product keeps ~16 bits of P), stored K-major as [head][key].
-//   5. O^T[512 x 32] = V^T . (P_hi + P_lo)^T        (4 dim chunks x 2 x 8
+//   5. O^T[512 x 16] = V^T . (P_hi + P_lo)^T        (4 dim chunks x 2 x 8
 //      MMAs; the V tile is read again as an MN-major operand)
 //   6. merge: each live tile writes its partial O into its own shared
 //      memory beside its per-head max m and sum l; after one cluster barrier
@@ -45,15 +45,17 @@ using namespace umma;
 namespace {
 
 constexpr int KT = 128;                     // keys per tile
-constexpr int HG = 32;                      // heads per CTA
+constexpr int HG = 16;                      // heads per CTA
 constexpr int THREADS = 512;
 constexpr int NTILES = ATT_SPLITS;          // 4 top-k tiles + the window = one cluster
-constexpr int KC = THREADS / HG;            // 16 chunks of 8 keys in the softmax
+constexpr int KC = THREADS / HG;            // softmax: chunks of KPT keys per head
+constexpr int KPT = KT / KC;                // keys per softmax thread
+constexpr int SCOLS = HG / 4;               // S^T columns each warp moves to the transpose
 constexpr int V_SLAB = KT * 128;            // 16 KB: 128 keys x 64 dims (bf16)
 constexpr int V_BYTES = 8 * V_SLAB;         // 128 KB
-constexpr int Q_SLAB = HG * 128;            // 4 KB: 32 heads x 64 dims
+constexpr int Q_SLAB = HG * 128;            // HG heads x 64 dims
 constexpr int Q_BYTES = 8 * Q_SLAB;         // 32 KB
-constexpr int P_SLAB = HG * 128;            // 4 KB: 32 heads x 64 keys
+constexpr int P_SLAB = HG * 128;            // HG heads x 64 keys
 constexpr int P_BYTES = 2 * P_SLAB;         // 8 KB
 constexpr int T_STRIDE = HG + 1;            // fp32 transpose row stride
 constexpr int T_BYTES = KT * T_STRIDE * 4;
@@ -62,8 +64,10 @@ constexpr size_t SMEM_BYTES = 1024 + T_OFF + T_BYTES;
 // The merge buffer [head][dim] (fp32) reuses the V tile once the second
 // product has completed.
 static_assert(HG * CSA2_LATENT * 4 <= V_BYTES, "merge buffer must fit the V tile");
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t S_COL = 0, O_COL = 32;   // S^T: 32 columns; O^T: 4 chunks x 32 columns
+constexpr uint32_t S_COL = 0, O_COL = 32;   // S^T: HG columns; O^T: 4 chunks x HG columns
+constexpr uint32_t TMEM_COLS = (O_COL + 4 * HG <= 128) ? 128 : 256;
+static_assert(HG == 16 || HG == 32, "head group of 16 or 32");
+static_assert(KPT == 4 || KPT == 8, "4 or 8 keys per softmax thread");
 constexpr uint32_t IDESC_S = idesc_f16(128, HG, true, false, false);
 constexpr uint32_t IDESC_O = idesc_f16(128, HG, true, true, false);
 
@@ -106,6 +110,23 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
     __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&a), y = *reinterpret_cast<__nv_bfloat162 *>(&b);
     __nv_bfloat162 r = __hmul2(x, y);
     return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// Tensor-memory load of as many columns as the array holds.
+template <int N>
+__device__ __forceinline__ void ld_cols(uint32_t a, uint32_t (&r)[N])
+{
+    if constexpr (N == 4) tmem_ld4(a, r);
+    else if constexpr (N == 8) tmem_ld8(a, r);
+    else if constexpr (N == 16) tmem_ld16(a, r);
+    else tmem_ld32(a, r);
+}
+// 2 or 4 packed bf16 pairs to shared memory.
+template <int N>
+__device__ __forceinline__ void st_pairs(uint8_t *p, const uint32_t (&v)[N])
+{
+    if constexpr (N == 2) *reinterpret_cast<uint2 *>(p) = make_uint2(v[0], v[1]);
+    else *reinterpret_cast<uint4 *>(p) = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t *err)
@@ -225,7 +246,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         mbar_init(&bar_s, 1);
         mbar_init(&bar_o, 4);                                // one commit per issuing warp
         mbar_fence_init();
-        // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x 32 heads, 128-byte
+        // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x HG heads, 128-byte
         // swizzled (K-major operand layout); heads past `heads` read as zero.
         mbar_arrive_expect_tx(&bar_q, Q_BYTES);
         for (int slab = 0; slab < 8; ++slab) tma_load_3d(Qs + slab * Q_SLAB, &map_q, 64 * slab, hg0, b, &bar_q);
@@ -236,7 +257,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     fence_after_sync();
     const uint32_t tb = tmem_base;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const int h = tid & (HG - 1), kc = tid >> 5;         // softmax: head, chunk of 8 keys
+    const int h = tid & (HG - 1), kc = tid / HG;         // softmax: head, chunk of KPT keys
 
     if (live) {
         // ---- 3. S^T = V . Q^T
@@ -255,20 +276,20 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         wait_bar(&bar_s, 0, c.error);
         fence_after_sync();
 
-        // ---- 4. softmax.  Scaled logits -> transpose (thread: key `row`, 8 heads).
+        // ---- 4. softmax.  Scaled logits -> transpose (thread: key `row`, SCOLS heads).
         {
-            uint32_t rr[8];
-            tmem_ld8(tb + lane_base + S_COL + 8 * (warp >> 2), rr);
+            uint32_t rr[SCOLS];
+            ld_cols(tb + lane_base + S_COL + SCOLS * (warp >> 2), rr);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                Ts[row * T_STRIDE + 8 * (warp >> 2) + j] = valid ? __uint_as_float(rr[j]) * scale : -INFINITY;
+            for (int j = 0; j < SCOLS; ++j)
+                Ts[row * T_STRIDE + SCOLS * (warp >> 2) + j] = valid ? __uint_as_float(rr[j]) * scale : -INFINITY;
         }
         __syncthreads();
         {
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, Ts[(8 * kc + j) * T_STRIDE + h]);
+            for (int j = 0; j < KPT; ++j) mx = fmaxf(mx, Ts[(KPT * kc + j) * T_STRIDE + h]);
             red_m[kc][h] = mx;
         }
         __syncthreads();
@@ -278,11 +299,11 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
             for (int r = 1; r < KC; ++r) m = fmaxf(m, red_m[r][h]);
             if (kc == 0) m_s[h] = m;
             float sum = 0.0f;
-            uint32_t hi[4], lo[4];
+            uint32_t hi[KPT / 2], lo[KPT / 2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float p0 = __expf(Ts[(8 * kc + 2 * i) * T_STRIDE + h] - m);
-                const float p1 = __expf(Ts[(8 * kc + 2 * i + 1) * T_STRIDE + h] - m);
+            for (int i = 0; i < KPT / 2; ++i) {
+                const float p0 = __expf(Ts[(KPT * kc + 2 * i) * T_STRIDE + h] - m);
+                const float p1 = __expf(Ts[(KPT * kc + 2 * i + 1) * T_STRIDE + h] - m);
                 sum += p0 + p1;
                 const __nv_bfloat162 ph = __floats2bfloat162_rn(p0, p1);
                 const float2 phf = __bfloat1622float2(ph);
@@ -290,10 +311,12 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
                 hi[i] = *reinterpret_cast<const uint32_t *>(&ph);
                 lo[i] = *reinterpret_cast<const uint32_t *>(&pl);
             }
-            // P^T row h, keys 8kc .. 8kc+7: slab kc/8, 16-byte chunk kc%8 (swizzled by h)
-            const uint32_t off = (kc >> 3) * P_SLAB + h * 128 + (((kc & 7) ^ (h & 7)) << 4);
-            *reinterpret_cast<uint4 *>(Ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(Pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            // P^T row h, keys KPT*kc ..: slab key/64, 16-byte chunk (key%64)/8
+            // swizzled by h, then the byte of the key inside its chunk
+            const int key0 = KPT * kc, k6 = key0 & 63;
+            const uint32_t off = (key0 >> 6) * P_SLAB + h * 128 + ((((k6 >> 3) ^ (h & 7))) << 4) + (k6 & 7) * 2;
+            st_pairs(Ph + off, hi);
+            st_pairs(Pl + off, lo);
             red_l[kc][h] = sum;
         }
         fence_proxy_async_smem();
@@ -311,7 +334,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
                     for (int kk = 0; kk < KT / 16; ++kk) {
                         const uint64_t ad = smem_desc(va + (2 * cc) * V_SLAB + kk * 2048, V_SLAB, 1024);
                         const uint64_t bd = smem_desc(pb + (kk >> 2) * P_SLAB + (kk & 3) * 32, 16, 1024);
-                        mma_ss(tb + O_COL + 32 * cc, ad, bd, IDESC_O, (part | kk) ? 1u : 0u);
+                        mma_ss(tb + O_COL + HG * cc, ad, bd, IDESC_O, (part | kk) ? 1u : 0u);
                     }
                 }
             }
@@ -339,8 +362,8 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     if (live) {
         wait_bar(&bar_o, 0, c.error);
         fence_after_sync();
-        uint32_t rr[32];
-        tmem_ld32(tb + lane_base + O_COL + 32 * (warp >> 2), rr);
+        uint32_t rr[HG];
+        ld_cols(tb + lane_base + O_COL + HG * (warp >> 2), rr);
         tmem_ld_wait();
         const int d = 128 * (warp >> 2) + 32 * (warp & 3) + lane;
 #pragma unroll
@@ -370,23 +393,23 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
     }
     __syncthreads();
     {
-        // This CTA's fifth (at most 820 float4, two per thread): every remote
-        // load of both is issued before any sum.
+        // This CTA's fifth of the HG x 512 outputs (NU float4 per thread):
+        // every remote load is issued before any sum.
         constexpr int total4 = HG * (CSA2_LATENT / 4);
-        static_assert((total4 + NTILES - 1) / NTILES <= 2 * THREADS, "two outputs per thread");
+        constexpr int NU = ((total4 + NTILES - 1) / NTILES + THREADS - 1) / THREADS;
         const int lo4 = tile * total4 / NTILES, hi4 = (tile + 1) * total4 / NTILES;
-        float4 v[2][NTILES];
+        float4 v[NU][NTILES];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NU; ++u) {
             const int i = lo4 + tid + u * THREADS;
 #pragma unroll
             for (int r = 0; r < NTILES; ++r)
                 v[u][r] = (i < hi4 && tile_live[r]) ? reinterpret_cast<const float4 *>(cluster.map_shared_rank(Ob, r))[i]
                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        float4 acc[2];
+        float4 acc[NU];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NU; ++u) {
             const int hh = min((lo4 + tid + u * THREADS) / (CSA2_LATENT / 4), HG - 1);
             acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -402,7 +425,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
         // wait for the others only after the output stores.
         asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NU; ++u) {
             const int i = lo4 + tid + u * THREADS;
             const int hh = i / (CSA2_LATENT / 4), d4 = i % (CSA2_LATENT / 4);
             if (i >= hi4 || hh >= nh) continue;
@@ -428,7 +451,7 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
 }
 
 // q viewed as a 3-D bf16 tensor (512 dims, heads, batch); boxes of 64 dims x
-// 32 heads, 128-byte swizzled.
+// HG heads, 128-byte swizzled.
 bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch)
 {
     auto fn = tensor_map_encoder();
