@@ -45,31 +45,35 @@ using namespace umma;
 namespace {
 
 constexpr int KT = 128;                     // keys per tile
-constexpr int HG = 16;                      // heads per CTA
 constexpr int THREADS = 512;
 constexpr int NTILES = ATT_SPLITS;          // 4 top-k tiles + the window = one cluster
-constexpr int KC = THREADS / HG;            // softmax: chunks of KPT keys per head
-constexpr int KPT = KT / KC;                // keys per softmax thread
-constexpr int SCOLS = HG / 4;               // S^T columns each warp moves to the transpose
 constexpr int V_SLAB = KT * 128;            // 16 KB: 128 keys x 64 dims (bf16)
 constexpr int V_BYTES = 8 * V_SLAB;         // 128 KB
-constexpr int Q_SLAB = HG * 128;            // HG heads x 64 dims
-constexpr int Q_BYTES = 8 * Q_SLAB;         // 32 KB
-constexpr int P_SLAB = HG * 128;            // HG heads x 64 keys
-constexpr int P_BYTES = 2 * P_SLAB;         // 8 KB
-constexpr int T_STRIDE = HG + 1;            // fp32 transpose row stride
-constexpr int T_BYTES = KT * T_STRIDE * 4;
-constexpr int Q_OFF = V_BYTES, PHI_OFF = Q_OFF + Q_BYTES, PLO_OFF = PHI_OFF + P_BYTES, T_OFF = PLO_OFF + P_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + T_OFF + T_BYTES;
-// The merge buffer [head][dim] (fp32) reuses the V tile once the second
-// product has completed.
-static_assert(HG * CSA2_LATENT * 4 <= V_BYTES, "merge buffer must fit the V tile");
 constexpr uint32_t S_COL = 0, O_COL = 32;   // S^T: HG columns; O^T: 4 chunks x HG columns
-constexpr uint32_t TMEM_COLS = (O_COL + 4 * HG <= 128) ? 128 : 256;
-static_assert(HG == 16 || HG == 32, "head group of 16 or 32");
-static_assert(KPT == 4 || KPT == 8, "4 or 8 keys per softmax thread");
-constexpr uint32_t IDESC_S = idesc_f16(128, HG, true, false, false);
-constexpr uint32_t IDESC_O = idesc_f16(128, HG, true, true, false);
+
+// Sizes for HG heads per CTA (16 or 32).
+template <int HG>
+struct Cfg {
+    static_assert(HG == 16 || HG == 32, "head group of 16 or 32");
+    static constexpr int KC = THREADS / HG;            // softmax: chunks of KPT keys per head
+    static constexpr int KPT = KT / KC;                // keys per softmax thread (4 or 8)
+    static constexpr int SCOLS = HG / 4;               // S^T columns each warp moves to the transpose
+    static constexpr int Q_SLAB = HG * 128;            // HG heads x 64 dims
+    static constexpr int Q_BYTES = 8 * Q_SLAB;
+    static constexpr int P_SLAB = HG * 128;            // HG heads x 64 keys
+    static constexpr int P_BYTES = 2 * P_SLAB;
+    static constexpr int T_STRIDE = HG + 1;            // fp32 transpose row stride
+    static constexpr int T_BYTES = KT * T_STRIDE * 4;
+    static constexpr int Q_OFF = V_BYTES, PHI_OFF = Q_OFF + Q_BYTES, PLO_OFF = PHI_OFF + P_BYTES,
+                         T_OFF = PLO_OFF + P_BYTES;
+    static constexpr size_t SMEM_BYTES = 1024 + T_OFF + T_BYTES;
+    // The merge buffer [head][dim] (fp32) reuses the V tile once the second
+    // product has completed.
+    static_assert(HG * CSA2_LATENT * 4 <= V_BYTES, "merge buffer must fit the V tile");
+    static constexpr uint32_t TMEM_COLS = (O_COL + 4 * HG <= 128) ? 128 : 256;
+    static constexpr uint32_t IDESC_S = idesc_f16(128, HG, true, false, false);
+    static constexpr uint32_t IDESC_O = idesc_f16(128, HG, true, true, false);
+};
 
 // Low and high bytes of the bf16 patterns of the 8 e2m1 magnitudes (0, .5,
 // 1, 1.5, 2, 3, 4, 6) as byte-permute tables: codes 0-3 in A, 4-7 in B.
@@ -136,14 +140,19 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
     return false;
 }
 
+template <int HG>
 __global__ void __cluster_dims__(NTILES, 1, 1) __launch_bounds__(THREADS, 1)
 attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads, const int32_t *topk, float scale,
                   void *out, int out_is_fp32, uint32_t flags, float *lse)
 {
+    using C = Cfg<HG>;
+    constexpr int KC = C::KC, KPT = C::KPT, SCOLS = C::SCOLS, Q_SLAB = C::Q_SLAB, Q_BYTES = C::Q_BYTES;
+    constexpr int P_SLAB = C::P_SLAB, T_STRIDE = C::T_STRIDE;
+    constexpr uint32_t TMEM_COLS = C::TMEM_COLS, IDESC_S = C::IDESC_S, IDESC_O = C::IDESC_O;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *Vs = sm, *Qs = sm + Q_OFF, *Ph = sm + PHI_OFF, *Pl = sm + PLO_OFF;
-    float *Ts = reinterpret_cast<float *>(sm + T_OFF);
+    uint8_t *Vs = sm, *Qs = sm + C::Q_OFF, *Ph = sm + C::PHI_OFF, *Pl = sm + C::PLO_OFF;
+    float *Ts = reinterpret_cast<float *>(sm + C::T_OFF);
     float *Ob = reinterpret_cast<float *>(Vs);
     __shared__ __align__(8) uint64_t bar_q, bar_s, bar_o;
     __shared__ uint32_t tmem_base;
@@ -451,40 +460,85 @@ attend_dsm_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int he
 }
 
 // q viewed as a 3-D bf16 tensor (512 dims, heads, batch); boxes of 64 dims x
-// HG heads, 128-byte swizzled.
-bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch)
+// hg heads, 128-byte swizzled.
+bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch, int hg)
 {
     auto fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[3] = {CSA2_LATENT, (cuuint64_t)heads, (cuuint64_t)batch};
     cuuint64_t strides[2] = {CSA2_LATENT * 2, (cuuint64_t)heads * CSA2_LATENT * 2};
-    cuuint32_t box[3] = {64, HG, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)hg, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)q, dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int HG>
+cudaError_t launch_hg(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale, void *out,
+                      int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse)
+{
+    CUtensorMap map_q;
+    if (!make_q_map(&map_q, q, heads, c.batch, HG)) return cudaErrorInvalidValue;
+    dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);
+    LaunchScope scope(CSA2_KERNEL_ATTEND, st);
+    return launch_pdl(attend_dsm_kernel<HG>, grid, dim3(THREADS), Cfg<HG>::SMEM_BYTES, st, map_q, c, heads, topk,
+                      scale, out, out_is_fp32, flags, lse);
+}
+
+// Clusters of the 16-head kernel the device runs at once (0 if unknown).
+int max_clusters_16()
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(NTILES, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg<16>::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = NTILES;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)attend_dsm_kernel<16>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    return n;
+}
+
 }  // namespace
 
+// 16-head CTAs halve each CTA's softmax, partial and merge work (the
+// latency of a small batch) but gather every key twice as often; they are
+// used while all their clusters run on the device at once (one wave),
+// 32-head CTAs beyond that.
 cudaError_t launch_attend_dsm(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
                               void *out, int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse)
 {
     static bool attr_done[64] = {};
+    static int wave16[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    int wave = dev < 64 ? wave16[dev] : 0;
     if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(attend_dsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        e = cudaFuncSetAttribute(attend_dsm_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg<16>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(attend_dsm_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)Cfg<32>::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
+        wave = max_clusters_16();
+        if (dev < 64) {
+            wave16[dev] = wave;
+            attr_done[dev] = true;
+        }
     }
-    CUtensorMap map_q;
-    if (!make_q_map(&map_q, q, heads, c.batch)) return cudaErrorInvalidValue;
-    dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);
-    LaunchScope scope(CSA2_KERNEL_ATTEND, st);
-    return launch_pdl(attend_dsm_kernel, grid, dim3(THREADS), SMEM_BYTES, st, map_q, c, heads, topk, scale, out,
-                      out_is_fp32, flags, lse);
+    const long long clusters16 = (long long)((heads + 15) / 16) * c.batch;
+    if (clusters16 <= wave) return launch_hg<16>(c, heads, q, topk, scale, out, out_is_fp32, flags, st, lse);
+    return launch_hg<32>(c, heads, q, topk, scale, out, out_is_fp32, flags, st, lse);
 }
 
 }  // namespace csa2
