@@ -105,8 +105,8 @@ def schedule_bytes(ws) -> dict:
 KNOWN_TRAFFIC = {
     "block_scan": {"bytes": 67_501_056 + 827_136, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
                    "sha256": "a3c2814836873bcbe6f19a489395cf2958005ce57066d43c01b840ceb548bc67"},
-    "attend": {"bytes": 1_560_320, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
-               "sha256": "9762f6cad1bf18be7ff484493bb488419c4bf06dabdd0bfe27644974904f3adf"},
+    "attend": {"bytes": 1_557_504, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
+               "sha256": "cd3023c6207320cb71394114629a30235262131d546683ca4df14f43dd616b84"},
 }
 
 
