@@ -256,8 +256,8 @@ def test_bad_page_id_sets_error():
 
 # ------------------------------------------------------------------ edge cases
 def test_empty_request_and_partial_head_group():
-    """A batch whose second request holds no tokens at all, with 40 heads (a
-    full 32-head group plus a partial one): the empty request gets an empty
+    """A batch whose second request holds no tokens at all, with 40 heads (two
+    full 16-head groups plus a partial one): the empty request gets an empty
     top-k and a zero output; the other matches the oracle."""
     w = synth.Workload("edge-B2-H40", 7, 2, 40, [3000, 0], [1, 1], "flat", ["full"], False, outliers=False)
     dw = DeviceWorkload(w, out_fp32=True)
@@ -273,6 +273,27 @@ def test_empty_request_and_partial_head_group():
     assert np.array_equal(top[0], rtop)
     r = refs[0].attend(bits(q[0]), top[0], SOFTMAX_SCALE)
     check_attention(dw.outs[0][0], r, "request 0, 40 heads")
+
+
+def test_partial_head_group_in_both_cta_shapes():
+    """40 heads in a batch small enough for 16-head attention CTAs (2
+    requests) and in one too large for a single wave of them (40 requests,
+    32-head CTAs: one full group and a partial one); sampled requests of
+    both against the oracle."""
+    for batch, picks in ((2, (0, 1)), (40, (0, 17, 39))):
+        w = synth.Workload(f"heads40-B{batch}", 9, batch, 40, [2500] * batch, [1] * batch, "flat", ["full"], False)
+        dw = DeviceWorkload(w, out_fp32=True)
+        dw.step()
+        torch.cuda.synchronize()
+        assert csa2.csa2_get_device_error(dw.cache) == 0
+        q, q_idx, hw = dw.layers[0]
+        for b in picks:
+            ref = OracleRequest(w, b, 2500)
+            top = dw.topk[0][b].cpu().numpy()
+            qb, wb = bits(q_idx[b]), hw[b].cpu().numpy()
+            check_swaps(top, oracle.index_flat(qb, wb, ref.keys8),
+                        lambda e: float(oracle.score_f64(qb, wb, ref.keys8[e:e + 1])[0]), f"B={batch} request {b}")
+            check_attention(dw.outs[0][b], ref.attend(bits(q[b]), top, SOFTMAX_SCALE), f"B={batch} request {b}")
 
 
 def test_reindex_layer_over_short_pool():
