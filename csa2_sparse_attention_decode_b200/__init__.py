@@ -32,7 +32,8 @@ INDEX_FLAT, INDEX_FULL, INDEX_REINDEX = 0, 1, 2
 EXPORTS = ("csa2_page_bytes", "csa2_swa_bytes", "csa2_workspace_bytes", "csa2_prefill", "csa2_append",
            "csa2_index", "csa2_attend", "csa2_get_device_error", "csa2_status_string", "csa2_set_profile_events",
            "csa2_launch_count", "csa2_attend_noalloc", "csa2_topk", "csa2_shard_blocks", "csa2_shard_pool",
-           "csa2_shard_rescore", "csa2_shard_topk", "csa2_attend_partial", "csa2_combine")
+           "csa2_shard_rescore", "csa2_shard_topk", "csa2_attend_partial", "csa2_combine",
+           "csa2_selftest_wait_timeout")
 MAX_SHARDS = 8
 ATTEND_NOALLOC_MAX_ROWS = 512
 KERNEL_BLOCK_SCORE, KERNEL_FLAT_SCORE, KERNEL_POOL_SCORE, KERNEL_SELECT, KERNEL_ATTEND, KERNEL_COMBINE = range(6)
@@ -80,6 +81,7 @@ def _load():
         "csa2_shard_topk": (C.c_int, [P, P, I32, P, P, P, P]),
         "csa2_attend_partial": (C.c_int, [P, I32, P, P, C.c_float, I32, P, P, C.c_uint32, P]),
         "csa2_combine": (C.c_int, [I32, P, P, I32, I32, P, I32, P]),
+        "csa2_selftest_wait_timeout": (C.c_int, [P, C.c_uint32, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -300,3 +302,9 @@ def csa2_combine(o_parts, lse_parts, out, stream=None):
     _check("csa2_combine", lib.csa2_combine(len(o_parts), po, pl, int(out.shape[0]), int(out.shape[1]), _ptr(out),
                                             fp32, _stream(stream)))
     del ko, kl
+
+
+def csa2_selftest_wait_timeout(error_word, polls: int = 1024, stream=None):
+    """Run the bounded-wait self-test: error_word (int32 device tensor of one
+    element) receives CSA2_DEV_TIMEOUT once the probe's wait runs out."""
+    _check("csa2_selftest_wait_timeout", lib.csa2_selftest_wait_timeout(_ptr(error_word), int(polls), _stream(stream)))

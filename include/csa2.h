@@ -362,6 +362,13 @@ typedef enum {
  * Pass NULLs to stop.  Process-wide setting; not thread-safe. */
 csa2_status csa2_set_profile_events(int32_t kernel, void *ev_start, void *ev_stop);
 
+/* Self-test of the bounded waits: launches one CTA that waits on a barrier
+ * nothing completes; after `polls` polls (1..65536) it gives up and writes
+ * CSA2_DEV_TIMEOUT to the device word *error_word (if it holds 0), as every
+ * kernel of the library does when a wait runs out.  Nothing faults or
+ * hangs.  For tests of the timeout reporting path. */
+csa2_status csa2_selftest_wait_timeout(int32_t *error_word, uint32_t polls, csa2_stream_t stream);
+
 /* Number of kernels this library has launched in this process so far. */
 uint64_t csa2_launch_count(void);
 

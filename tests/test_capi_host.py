@@ -121,3 +121,10 @@ def test_sharded_calls_reject_invalid_arguments_before_launch(csa2):
     assert L.csa2_combine(2, lp, lp, 0, 64, good, 0, None) == 1
     assert L.csa2_combine(2, lp, lp, 2, 129, good, 0, None) == 1
     assert L.csa2_combine(2, C.cast(mis, C.c_void_p), lp, 2, 64, good, 0, None) == 1
+
+
+def test_selftest_wait_timeout_rejects_invalid_arguments(csa2):
+    L = csa2.lib
+    assert L.csa2_selftest_wait_timeout(None, 100, None) == 1
+    assert L.csa2_selftest_wait_timeout(C.c_void_p(256 * 100), 0, None) == 1
+    assert L.csa2_selftest_wait_timeout(C.c_void_p(256 * 100), (1 << 16) + 1, None) == 1

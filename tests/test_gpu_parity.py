@@ -254,6 +254,21 @@ def test_bad_page_id_sets_error():
     assert csa2.csa2_get_device_error(dw.cache) == 1
 
 
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait that nothing completes gives up after its poll limit and
+    reports CSA2_DEV_TIMEOUT through the error word; later work still runs."""
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa2.csa2_selftest_wait_timeout(err, 256)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 5                       # CSA2_DEV_TIMEOUT
+    csa2.csa2_selftest_wait_timeout(err, 256)         # the first code stays
+    w = synth.workload(0, small=True)
+    dw = DeviceWorkload(w, out_fp32=True)
+    dw.step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_get_device_error(dw.cache) == 0 and int(err.item()) == 5
+
+
 # ------------------------------------------------------------------ edge cases
 def test_empty_request_and_partial_head_group():
     """A batch whose second request holds no tokens at all, with 40 heads (two
