@@ -311,6 +311,15 @@ def test_partial_head_group_in_both_cta_shapes():
             check_attention(dw.outs[0][b], ref.attend(bits(q[b]), top, SOFTMAX_SCALE), f"B={batch} request {b}")
 
 
+def test_maximum_heads():
+    """128 query heads, the most csa2_attend takes (eight 16-head groups per
+    request), with Full and Reuse layers, against the oracle."""
+    w = synth.Workload("heads128-B2", 13, 2, 128, [6000, 3001], [1, 2], "hier", ["full", "reuse"], False)
+    dw = DeviceWorkload(w, out_fp32=True)
+    refs = [OracleRequest(w, b, w.n_tok[b]) for b in range(w.batch)]
+    check_step(w, dw, refs)
+
+
 def test_reindex_layer_over_short_pool():
     """A request short enough that its pool is every entry (fewer than 2048
     blocks): Full and Reindex both select from it exactly."""

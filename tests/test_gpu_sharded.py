@@ -70,7 +70,7 @@ def _run_and_check(w, n_shards, out_fp32=True):
             check_attention(ls.outs[li][b], r, f"req {b} layer {li} ({n_shards} shards)")
 
 
-@pytest.mark.parametrize("n_shards", [1, 2, 3, 4])
+@pytest.mark.parametrize("n_shards", [1, 2, 3, 4, 8])
 def test_reuse_group_sharded_matches_oracle(n_shards):
     # 2 requests x 24,000 entries: 3,000 blocks, so the block top-2048 prunes
     _run_and_check(synth.workload(3, small=True), n_shards)
