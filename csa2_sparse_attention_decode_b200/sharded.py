@@ -220,17 +220,33 @@ class LocalShards:
 
 class DistShard:
     """This rank's shard of a sharded decode; `ops` has the stage methods of
-    Shard.  Every rank runs the same collectives in the same order."""
+    Shard.  Every rank runs the same collectives in the same order: one
+    all-gather per exchange, with the exchanged tensors packed into one
+    flat 32-bit buffer (ids beside the bit patterns of their scores, the
+    output beside its log-sum-exp), so a Full layer makes three."""
 
     def __init__(self, ops, layers: Sequence[str], group=None):
         import torch.distributed as dist
         self.dist, self.ops, self.layers, self.group = dist, ops, list(layers), group
         self.world = dist.get_world_size(group)
 
-    def _all_gather(self, t: torch.Tensor) -> List[torch.Tensor]:
-        out = [torch.empty_like(t) for _ in range(self.world)]
-        self.dist.all_gather(out, t.contiguous(), group=self.group)
-        return out
+    def _exchange(self, parts: Sequence[torch.Tensor]) -> List[List[torch.Tensor]]:
+        """All-gather of 32-bit tensors packed end to end; returns, per rank,
+        views of that rank's copies in the original shapes and dtypes."""
+        # every part starts on a 16-byte boundary (4 words), so each view is
+        # aligned for its dtype and for the library's vector loads
+        words, spans = [], []
+        for p in parts:
+            w = p.contiguous().view(torch.int32).reshape(-1)
+            spans.append((sum(x.numel() for x in words), w.numel()))
+            words.append(w)
+            if w.numel() % 4:
+                words.append(torch.zeros(4 - w.numel() % 4, dtype=torch.int32, device=w.device))
+        flat = torch.cat(words)
+        out = torch.empty(self.world * flat.numel(), dtype=torch.int32, device=flat.device)
+        self.dist.all_gather_into_tensor(out, flat, group=self.group)
+        return [[out[r * flat.numel() + o: r * flat.numel() + o + n].view(p.dtype).view(p.shape)
+                 for p, (o, n) in zip(parts, spans)] for r in range(self.world)]
 
     def step(self, inputs, outs, scale: float, stream=None):
         """inputs[layer] = (q, q_idx, w); outs[layer] receives the combined
@@ -238,11 +254,11 @@ class DistShard:
         for li, mode, grp in _schedule(self.layers):
             q, q_idx, hw = inputs[li]
             if mode == "full":
-                ids, sc = self.ops.blocks(q_idx, hw, stream)
-                self.ops.pool_from(self._all_gather(ids), self._all_gather(sc), stream)
+                got = self._exchange(self.ops.blocks(q_idx, hw, stream))
+                self.ops.pool_from([g[0] for g in got], [g[1] for g in got], stream)
             if mode in ("full", "reindex"):
-                ids, sc = self.ops.rescore(q_idx, hw, stream)
-                self.ops.topk_from(grp, self._all_gather(ids), self._all_gather(sc), stream)
+                got = self._exchange(self.ops.rescore(q_idx, hw, stream))
+                self.ops.topk_from(grp, [g[0] for g in got], [g[1] for g in got], stream)
             flags = ATTEND_INPUTS_SETTLED if mode == "reuse" else 0
-            o, lse = self.ops.attend(grp, q, scale, flags, stream)
-            self.ops.combine(self._all_gather(o), self._all_gather(lse), outs[li], stream)
+            got = self._exchange(self.ops.attend(grp, q, scale, flags, stream))
+            self.ops.combine([g[0] for g in got], [g[1] for g in got], outs[li], stream)

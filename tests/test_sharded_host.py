@@ -192,3 +192,40 @@ def test_dist_sharded_step_equals_unsharded_oracle(world, n_tok, m):
         assert res["tops"][layer_group[li]] == ref_top, f"layer {li}"
         # output: the merge of the shards' attention = attention over all keys
         assert np.allclose(res["outs"][li], ref_out, rtol=1e-11, atol=1e-12), f"layer {li}"
+
+
+def _exchange_rank(rank, world, port, q):
+    try:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        from csa2_sparse_attention_decode_b200.sharded import DistShard
+        ds = DistShard(None, [], None)
+        ids = torch.arange(3, dtype=torch.int32) + 10 * rank
+        sc = torch.tensor([0.5, -2.0], dtype=torch.float32) * (rank + 1)
+        o = torch.full((2, 3), float(rank), dtype=torch.float64)
+        got = ds._exchange([ids, sc, o])
+        ok = all(torch.equal(got[r][0], torch.arange(3, dtype=torch.int32) + 10 * r) and
+                 torch.equal(got[r][1], torch.tensor([0.5, -2.0]) * (r + 1)) and
+                 torch.equal(got[r][2], torch.full((2, 3), float(r), dtype=torch.float64)) and
+                 all((got[r][i].data_ptr() - got[0][0].data_ptr()) % 16 == 0 for i in range(3))
+                 for r in range(world))
+        dist.destroy_process_group()
+        q.put((rank, ok, None))
+    except Exception:
+        import traceback
+        q.put((rank, False, traceback.format_exc()))
+
+
+def test_dist_exchange_packs_mixed_parts_in_one_all_gather():
+    # int32 ids (3 words), float32 scores (2) and a float64 block (12) come
+    # back per rank in their own shapes and dtypes, every part 16-byte aligned
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_exchange_rank, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(ok for _, ok, _ in got), [e for _, _, e in got if e]
