@@ -30,7 +30,7 @@ from typing import List, Sequence
 
 import torch
 
-from . import (ATTEND_INPUTS_SETTLED, KERNEL_ATTEND, MAX_BLOCKS, PAGE_ENTRIES, POOL, SWA, TOPK, Cache, csa2_append,
+from . import (ATTEND_INPUTS_SETTLED, KERNEL_ATTEND, MAX_BLOCKS, MAX_SHARDS, PAGE_ENTRIES, POOL, SWA, TOPK, Cache, csa2_append,
                csa2_attend_partial, csa2_cache, csa2_combine, csa2_set_profile_events, csa2_shard_blocks,
                csa2_shard_pool, csa2_shard_rescore, csa2_shard_topk, workspace)
 
@@ -164,6 +164,10 @@ class LocalShards:
     def __init__(self, dw, n_shards: int, out_fp32: bool = False):
         from .harness import SOFTMAX_SCALE
         w = dw.w
+        if w.index != "hier":
+            raise ValueError("the sharded step runs the hierarchical indexer; this workload indexes flat")
+        if not 1 <= n_shards <= MAX_SHARDS:
+            raise ValueError(f"1..{MAX_SHARDS} shards")
         self.dw, self.n_shards, self.scale = dw, n_shards, SOFTMAX_SCALE
         n_tok = dw.cache.n_tokens.cpu().tolist()
         offs = [shard_offsets(t // m, t, m, n_shards) for t, m in zip(n_tok, w.m)]
