@@ -171,7 +171,7 @@ def _rank(rank, world, port, n_tok, m, q):
         q.put((rank, None, traceback.format_exc()))
 
 
-@pytest.mark.parametrize("world,n_tok,m", [(2, 24000, 1), (3, 40002, 2), (2, 80000, 1)])
+@pytest.mark.parametrize("world,n_tok,m", [(2, 24000, 1), (3, 40002, 2), (2, 80000, 1), (4, 40001, 2)])
 def test_dist_sharded_step_equals_unsharded_oracle(world, n_tok, m):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
