@@ -300,6 +300,9 @@ def test_hierarchical_pool_structure():
     exp_pool = np.concatenate([np.arange(b * 8, min(b * 8 + 8, n)) for b in blocks])
     assert plen == exp_pool.size and np.array_equal(pool[:plen], exp_pool)
     assert set(top.tolist()) <= set(exp_pool.tolist()) and (top >= 0).all()
+    # both selections against a brute-force sort (score desc, lower id first)
+    assert list(blocks) == _brute_topk(bs, 2048)
+    assert list(top) == _brute_topk(oracle.score_f32(q, w, keys8[exp_pool]), 512, exp_pool)
 
 
 # ------------------------------------------------------------------ P5 / P7: attention
@@ -414,3 +417,93 @@ def test_lse_combine_of_a_key_split_is_the_whole_attention():
     assert not z.any()
     # a dropped weight (plain mean of the parts) is detectably wrong
     assert not np.allclose(o_parts[[0, 1, 3]].mean(0), whole, atol=1e-6)
+
+
+# ------------------------------------------------------------------ entry building: which tokens, which gate
+def _fp8_bytes(x) -> np.ndarray:
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_build_entries_pairs_tokens_and_shares_each_tokens_gate():
+    """m = 2 ([blog-0539] §1: m tokens become one entry; [nxbn] §4.2, gated
+    compression with one gate logit per token, shared by latent and key).
+    Entry e must come from tokens 2e and 2e+1 with gates g[2e], g[2e+1].
+    Gate pairs that differ by 40 make the entry exactly the dominant token
+    (closed form), and equal gates make it the one-rounding mean; the mode
+    varies per entry, so a shifted pairing, a gate taken from the wrong token
+    or a key compressed without the gate all change some entry's bytes."""
+    rng = np.random.default_rng(11)
+    n_ent, e_begin = 12, 5                      # tokens [10, 34) of a request
+    lat = (rng.standard_normal((2 * n_ent, 512)) * 2).astype(np.float32)
+    key = rng.standard_normal((2 * n_ent, 128)).astype(np.float32)
+    gate = np.zeros(2 * n_ent, np.float32)
+    modes = [0, 1, 2, 1, 0, 2, 0, 0, 1, 1, 2, 0]
+    for e, mode in enumerate(modes):
+        base = np.float32(rng.standard_normal())
+        if mode == 0:
+            gate[2 * e], gate[2 * e + 1] = base + 20, base - 20     # first token dominates
+        elif mode == 1:
+            gate[2 * e], gate[2 * e + 1] = base - 20, base + 20     # second token dominates
+        else:
+            gate[2 * e] = gate[2 * e + 1] = base                    # equal weights
+    codes, scales, keys8 = oracle.build_entries(2, lat, key, gate, e_begin=e_begin)
+    assert codes.shape == (n_ent, 256) and keys8.shape == (n_ent, 128)
+    for e, mode in enumerate(modes):
+        if mode == 2:
+            want_lat = ((lat[2 * e].astype(np.float64) + lat[2 * e + 1]) / 2).astype(np.float32)
+            want_key = ((key[2 * e].astype(np.float64) + key[2 * e + 1]) / 2).astype(np.float32)
+        else:
+            want_lat, want_key = lat[2 * e + mode], key[2 * e + mode]
+        c, s = oracle.pack_latent(want_lat)
+        assert np.array_equal(codes[e], c) and np.array_equal(scales[e], s), (e, mode)
+        assert np.array_equal(keys8[e], _fp8_bytes(want_key)), (e, mode)
+    # m = 1: entry e is token e, whatever its gate
+    c1, s1, k1 = oracle.build_entries(1, lat[:7], key[:7], gate[:7] * 0 + 30, e_begin=3)
+    for e in range(7):
+        c, s = oracle.pack_latent(lat[e])
+        assert np.array_equal(c1[e], c) and np.array_equal(s1[e], s)
+        assert np.array_equal(k1[e], _fp8_bytes(key[e]))
+
+
+def test_build_summaries_counts_a_ragged_last_block():
+    """Block summary = mean of the indexer keys of the (up to 8) entries
+    present in the block ([blog-0539] §3, hierarchical blocks of 8
+    positions).  With N = 8*5 + 3 the last block holds c = 3 entries: its
+    summary is torch's e4m3 of the exact mean of those three keys, and every
+    full block's the mean of its eight."""
+    rng = np.random.default_rng(12)
+    n = 8 * 5 + 3
+    keys8 = oracle.e4m3_encode((rng.standard_normal((n, 128)) * 4).astype(np.float32))
+    kv = oracle.e4m3_decode(keys8)
+    summ = oracle.build_summaries(keys8)
+    assert summ.shape == (6, 128)
+    for b in range(6):
+        rows = kv[8 * b:min(n, 8 * b + 8)]
+        assert rows.shape[0] == (3 if b == 5 else 8)
+        mean = (rows.sum(0) / rows.shape[0]).astype(np.float32)
+        assert np.array_equal(summ[b], _fp8_bytes(mean)), b
+    # a divisor of 8 (or of anything but 3) would change the last block
+    wrong = _fp8_bytes((kv[40:43].sum(0) / 8).astype(np.float32))
+    assert not np.array_equal(summ[5], wrong)
+
+
+def test_swa_window_slot_placement():
+    """The SWA ring ([blog-0539] §3: swa_window_size 128, FP8) holds token
+    position p in slot p mod 128, and min(n_tok, 128) slots are valid.
+    n_tok = 300: slot s holds token 256 + s for s < 44 and token 128 + s for
+    s >= 44.  n_tok = 50: slots 0..49 hold tokens 0..49, the rest are empty."""
+    rng = np.random.default_rng(13)
+    toks = (rng.standard_normal((300, 512)) * np.exp(rng.standard_normal((300, 1)))).astype(np.float32)
+    codes, scale, nv = oracle.swa_window(toks[300 - 128:], 300)
+    assert nv == 128
+    for s in range(128):
+        t = 256 + s if s < 44 else 128 + s
+        c, sc = oracle.swa_quant(toks[t])
+        assert scale[s] == sc[0] and np.array_equal(codes[s], c[0]), s
+        assert scale[s] == 2.0 ** math.ceil(math.log2(np.abs(toks[t]).max() / 448.0))
+    codes, scale, nv = oracle.swa_window(toks[:50], 50)
+    assert nv == 50
+    for s in range(50):
+        c, sc = oracle.swa_quant(toks[s])
+        assert scale[s] == sc[0] and np.array_equal(codes[s], c[0]), s
+    assert not codes[50:].any() and not scale[50:].any()
