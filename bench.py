@@ -12,9 +12,10 @@ replayed; each timed replay is bracketed by CUDA events, with a 256 MB write
 between replays to flush L2.  Under torchrun every rank runs its own replica
 (weak scaling) and the slowest rank's time counts.
 
---impl reference times the CPU oracle (plain C, one thread) on the host,
-round-robin over the stages of one request's step, and reports the same
-metric; it runs on rank 0 only.
+--impl reference times the CPU oracle (plain C) on the host cores: each step
+is the whole batch's decode step, requests on threads of their own and each
+scan's chunks spread over one thread per core; it reports the same metric and
+runs on rank 0 only.
 """
 from __future__ import annotations
 
@@ -134,56 +135,94 @@ def measured_peak_hbm():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
-    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """SM clocks and clock-event (throttle) reasons, sampled about every
+    millisecond through NVML from a background thread (nvidia-smi's 50 ms
+    loop as a fallback).  Started before warm-up; mark() brackets the timed
+    region, whose samples are summarised on their own beside the whole run's."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples = []                     # (perf_counter, sm_mhz, sm_max_mhz, reasons)
+        self.window = [None, None]
+        self._stop = threading.Event()
+        self.thread = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.device)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(
+                f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0")
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(p.uuid))
+
+    def _run_nvml(self, nv, h):
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        masks = [(n, getattr(nv, c)) for n, c in self.REASONS]
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                break
+            self.samples.append((time.perf_counter(), float(mhz), float(smax),
+                                 tuple(n for n, m in masks if r & m)))
+            time.sleep(0.001)
+
+    def _run_smi(self, idx):
+        q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        proc = subprocess.Popen(["nvidia-smi", f"--id={idx}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        for line in proc.stdout:
+            if self._stop.is_set():
+                break
+            parts = [x.strip() for x in line.split(",")]
+            try:
+                self.samples.append((time.perf_counter(), float(parts[0]), float(parts[1]),
+                                     tuple(n for (n, _), v in zip(self.REASONS, parts[2:6])
+                                           if v.lower().startswith("active"))))
+            except (ValueError, IndexError):
+                continue
+        proc.terminate()
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            nv, h = self._nvml_handle()
+            self.source = "nvml, ~1 ms"
+            self.thread = threading.Thread(target=self._run_nvml, args=(nv, h), daemon=True)
         except Exception:
-            self.proc = None
+            self.source = "nvidia-smi, 50 ms"
+            self.thread = threading.Thread(target=self._run_smi, args=(self.device.index or 0,), daemon=True)
+        self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def mark(self, which: int):
+        self.window[which] = time.perf_counter()
+
+    @staticmethod
+    def _summary(rows):
+        sm = [r[1] for r in rows]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(r[2] for r in rows) if rows else None,
+                "reasons": sorted({n for r in rows for n in r[3]}), "samples": len(rows)}
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.t.join(timeout=2)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        rows = list(self.samples)
+        t0, t1 = self.window
+        timed = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        out = self._summary(timed)
+        out["source"] = self.source or "unavailable"
+        out["whole_run"] = self._summary(rows)
+        return out
 
 
 def bench_config(w: synth.Workload) -> dict:
@@ -195,9 +234,29 @@ def bench_config(w: synth.Workload) -> dict:
 
 
 # ------------------------------------------------------------------ oracle (CPU) side
+def host_cpu() -> dict:
+    """Host cores available to this process and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return {"nproc": n, "cpu_model": model}
+
+
 class OracleQuery:
-    """The oracle's decode step for one request of workload w, split into
-    stage units so it can be timed in bounded slices."""
+    """The oracle's decode step for one request of workload w, as a list of
+    stages run in order; the callables of one stage are independent of one
+    another (the block or key scan's chunks), so a pool may run them at once.
+    The oracle's calls are C through ctypes, which releases the GIL."""
 
     CHUNK = 4096
 
@@ -228,87 +287,135 @@ class OracleQuery:
             q, qi, hw = synth.queries(w, li)
             self.layers.append((q[b].view(torch.int16).numpy().view(np.uint16),
                                 qi[b].view(torch.int16).numpy().view(np.uint16), hw[b].numpy()))
-        self.units = self._units()
+        self.stages = self._stages()
 
-    def _units(self):
-        """List of callables; running all of them in order is one full step."""
+    def _stages(self):
+        """List of stages (lists of callables); running them in order is one
+        full step."""
         w, o = self.w, self.o
         st = {}
-        units = []
+        stages = []
         nb = self.summ.shape[0]
         n_ent = self.keys8.shape[0]
         for li, mode in enumerate(w.layers):
             q, qi, hw = self.layers[li]
             if mode == "full" and w.index == "flat":
                 st_scores = np.empty(n_ent, np.float32)
-                for c0 in range(0, n_ent, self.CHUNK):
-                    units.append(lambda c0=c0, qi=qi, hw=hw, s=st_scores:
-                                 s.__setitem__(slice(c0, c0 + self.CHUNK),
-                                               o.score_f32(qi, hw, self.keys8[c0:c0 + self.CHUNK])))
-                units.append(lambda s=st_scores: st.__setitem__("top", o.topk(s, 512)))
+                stages.append([lambda c0=c0, qi=qi, hw=hw, s=st_scores:
+                               s.__setitem__(slice(c0, c0 + self.CHUNK),
+                                             o.score_f32(qi, hw, self.keys8[c0:c0 + self.CHUNK]))
+                               for c0 in range(0, n_ent, self.CHUNK)])
+                stages.append([lambda s=st_scores: st.__setitem__("top", o.topk(s, 512))])
             elif mode == "full":
                 bsc = np.empty(nb, np.float32)
-                for c0 in range(0, nb, self.CHUNK):
-                    units.append(lambda c0=c0, qi=qi, hw=hw, s=bsc:
-                                 s.__setitem__(slice(c0, c0 + self.CHUNK),
-                                               o.score_f32(qi, hw, self.summ[c0:c0 + self.CHUNK])))
+                stages.append([lambda c0=c0, qi=qi, hw=hw, s=bsc:
+                               s.__setitem__(slice(c0, c0 + self.CHUNK),
+                                             o.score_f32(qi, hw, self.summ[c0:c0 + self.CHUNK]))
+                               for c0 in range(0, nb, self.CHUNK)])
 
                 def pool_unit(s=bsc):
                     blocks = o.topk(s, 2048)
                     st["pool"], st["plen"] = o.expand_pool(blocks, n_ent)
-                units.append(pool_unit)
-                units.append(lambda qi=qi, hw=hw: st.__setitem__(
-                    "top", o.index_pool(qi, hw, self.keys8, st["pool"], st["plen"])))
+                stages.append([pool_unit])
+                stages.append([lambda qi=qi, hw=hw: st.__setitem__(
+                    "top", o.index_pool(qi, hw, self.keys8, st["pool"], st["plen"]))])
             elif mode == "reindex":
-                units.append(lambda qi=qi, hw=hw: st.__setitem__(
-                    "top", o.index_pool(qi, hw, self.keys8, st["pool"], st["plen"])))
+                stages.append([lambda qi=qi, hw=hw: st.__setitem__(
+                    "top", o.index_pool(qi, hw, self.keys8, st["pool"], st["plen"]))])
 
             def attend_unit(q=q):
                 ids = st["top"][st["top"] >= 0]
                 st["out"] = o.attend(q, self.codes[ids], self.scales[ids], self.win[0], self.win[1],
                                      1.0 / math.sqrt(512.0))
-            units.append(attend_unit)
-        return units
+            stages.append([attend_unit])
+        return stages
 
-    def run_full(self):
-        for u in self.units:
-            u()
+    def run_full(self, pool=None):
+        """One full step; with a thread pool each stage's callables run at once."""
+        for stage in self.stages:
+            if pool is None or len(stage) == 1:
+                for u in stage:
+                    u()
+            else:
+                for f in [pool.submit(u) for u in stage]:
+                    f.result()
 
 
-def cpu_baseline(w: synth.Workload, repeats: int = 4) -> dict:
-    q = OracleQuery(w, 0)
-    q.run_full()
-    t0 = time.perf_counter()
-    for _ in range(repeats):
-        q.run_full()
-    dt = time.perf_counter() - t0
-    return {"value": repeats / dt, "unit": "queries/s", "cores": 1, "kind": "oracle",
-            "sample": f"{repeats} x one request's full step ({w.name}, request 0, {len(q.units)} stages), "
-                      f"single-threaded C oracle"}
+class OracleBatch:
+    """The oracle's decode step for every request of a workload.  step()
+    runs the requests concurrently, one host thread each, and their scan
+    chunks on a pool of one thread per host core."""
+
+    def __init__(self, w: synth.Workload):
+        import concurrent.futures as cf
+        self.w = w
+        self.cpu = host_cpu()
+        self.threads = max(1, self.cpu["nproc"])
+        self.chunk_pool = cf.ThreadPoolExecutor(self.threads)
+        self.req_pool = cf.ThreadPoolExecutor(w.batch)
+        self.queries = list(self.req_pool.map(lambda b: OracleQuery(w, b), range(w.batch)))
+
+    def step(self):
+        for f in [self.req_pool.submit(q.run_full, self.chunk_pool) for q in self.queries]:
+            f.result()
+
+    def close(self):
+        self.chunk_pool.shutdown()
+        self.req_pool.shutdown()
+
+
+def cpu_baseline(w: synth.Workload, repeats: int = 2) -> dict:
+    """The oracle on this host: the whole batch's step on all host cores
+    (the value), and one request's step on one thread (beside it)."""
+    ob = OracleBatch(w)
+    try:
+        q0 = ob.queries[0]
+        q0.run_full()
+        t0 = time.perf_counter()
+        q0.run_full()
+        single = 1.0 / (time.perf_counter() - t0)
+        ob.step()
+        t0 = time.perf_counter()
+        for _ in range(repeats):
+            ob.step()
+        dt = time.perf_counter() - t0
+    finally:
+        ob.close()
+    return {"value": w.batch * repeats / dt, "unit": "queries/s", "cores": ob.threads, "kind": "oracle",
+            "cpu_model": ob.cpu["cpu_model"], "nproc": ob.cpu["nproc"],
+            "sample": f"{repeats} whole steps of {w.name} ({w.batch} requests x {sum(len(q) for q in q0.stages)} "
+                      f"stage units): requests on {w.batch} threads at once, each stage's scan chunks on a pool "
+                      f"of {ob.threads} threads (one per host core); plain C oracle through ctypes",
+            "single_thread": {"value": single, "unit": "queries/s", "cores": 1,
+                              "sample": f"one request's full step ({w.name}, request 0) on one thread"}}
 
 
 def run_reference(args, w: synth.Workload, rank: int, world: int):
+    """The oracle arm: each step is the whole batch's decode step (the GPU
+    arm's unit of work) on all host cores."""
     if rank != 0:
         return
-    q = OracleQuery(w, 0)
-    U = len(q.units)
-    k = 0
-    for _ in range(args.warmup):
-        q.units[k % U]()
-        k += 1
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        q.units[k % U]()
-        k += 1
-    dt = time.perf_counter() - t0
-    value = (args.steps / U) / dt
+    ob = OracleBatch(w)
+    try:
+        for _ in range(args.warmup):
+            ob.step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            ob.step()
+        dt = time.perf_counter() - t0
+    finally:
+        ob.close()
+    value = w.batch * args.steps / dt
+    units = sum(len(s) for s in ob.queries[0].stages)
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * dt / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": bench_config(w), "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
-                             "sample": f"each step = one of the {U} stage units of one request's decode step "
-                                       f"(round-robin; {U} steps = one query)"},
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": ob.threads, "kind": "oracle",
+                             "cpu_model": ob.cpu["cpu_model"], "nproc": ob.cpu["nproc"],
+                             "sample": f"each step = the whole batch's decode step ({w.batch} requests x {units} "
+                                       f"stage units), requests on {w.batch} threads at once and each stage's "
+                                       f"scan chunks on {ob.threads} threads"},
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -482,6 +589,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     k_att = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     n_layers = rn.n_layers
 
+    # clocks are sampled from here on, through warm-up, the timed region and
+    # the end-to-end loop
+    sampler = ClockSampler(dev)
+    sampler.start()
     # warm up eagerly once (first-call attribute set-up happens outside capture)
     with torch.cuda.stream(stream):
         rn.restore(stream)
@@ -525,11 +636,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         one(i)
     stream.synchronize()
 
-    sampler = ClockSampler(local_rank)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
+    sampler.mark(0)
     step_ms, scan_ms, att_ms = [], [], []
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
     for i in range(args.steps):
@@ -542,7 +652,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
+    sampler.mark(1)
     max_total_ms = max_over_ranks(sum(step_ms), world, dev)
     value = job_throughput(world, rn.batch, args.steps, max_total_ms)
 
@@ -603,6 +713,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     e2e_ms = [t0.elapsed_time(t1)]
     e2e_value = job_throughput(world, rn.batch, e2e_steps, max_over_ranks(sum(e2e_ms), world, dev))
     del slot_graphs
+    clocks = sampler.stop()
 
     # ---- roofline: attention (the largest share of the step's kernel time)
     # and the index scan, both timed live with CUDA events on the launching

@@ -55,11 +55,9 @@ extern "C" csa2_status csa2_attend_noalloc(const csa2_cache *cache, int32_t head
                                            const int32_t *topk, float scale, void *out, int32_t out_is_fp32,
                                            csa2_stream_t stream)
 {
-    if (!cache || !cache->pool || !cache->page_table || !cache->n_tokens || !cache->m || !cache->swa ||
-        !cache->pending || !cache->error)
-        return CSA2_ERR_INVALID_ARG;
-    if (cache->batch <= 0 || cache->n_pages <= 0 || cache->max_pages <= 0) return CSA2_ERR_INVALID_ARG;
-    if (!aligned_to(cache->pool, 256) || !aligned_to(cache->swa, 256)) return CSA2_ERR_INVALID_ARG;
+    CSA2_TRACE("csa2_attend_noalloc");
+    const csa2_status st = csa2::check_cache(cache);
+    if (st != CSA2_OK) return st;
     if (heads <= 0 || heads > 128 || !q || !topk || !out || !aligned_to(out, 16) || !aligned_to(q, 16))
         return CSA2_ERR_INVALID_ARG;
     // The fixed array holds the partials of at most this many (request, head) rows.

@@ -407,15 +407,15 @@ bool make_q_map(CUtensorMap *m, const uint16_t *q, int heads, int batch)
 cudaError_t launch_attend_umma(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
                                void *out, int out_is_fp32, uint32_t flags, float *part_o, cudaStream_t st)
 {
-    static bool attr_done[64] = {};
+    static DeviceOnce once;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = once.run(dev, [] {
+            return cudaFuncSetAttribute(attend_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)SMEM_BYTES);
+        });
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(attend_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
-    }
     CUtensorMap map_q;
     if (!make_q_map(&map_q, q, heads, c.batch)) return cudaErrorInvalidValue;
     dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);

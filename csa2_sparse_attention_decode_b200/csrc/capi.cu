@@ -31,6 +31,17 @@ void csa2::note_launch(int kernel, cudaStream_t st, bool before)
         cudaEventRecord(ev, st);
 }
 
+csa2_status csa2::check_cache(const csa2_cache *c)
+{
+    auto al = [](const void *p, size_t a) { return ((uintptr_t)p % a) == 0; };
+    if (!c || !c->pool || !c->page_table || !c->n_tokens || !c->m || !c->swa || !c->pending || !c->error)
+        return CSA2_ERR_INVALID_ARG;
+    if (c->batch <= 0 || c->n_pages <= 0 || c->max_pages <= 0) return CSA2_ERR_INVALID_ARG;
+    if ((int64_t)c->max_pages * CSA2_PAGE_ENTRIES > (int64_t)1 << 30) return CSA2_ERR_INVALID_ARG;
+    if (!al(c->pool, 256) || !al(c->swa, 256) || !al(c->pending, 16)) return CSA2_ERR_INVALID_ARG;
+    return CSA2_OK;
+}
+
 namespace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -62,16 +73,6 @@ Workspace layout(void *base, int32_t batch, int32_t heads, int32_t max_entries)
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-csa2_status check_cache(const csa2_cache *c)
-{
-    if (!c || !c->pool || !c->page_table || !c->n_tokens || !c->m || !c->swa || !c->pending || !c->error)
-        return CSA2_ERR_INVALID_ARG;
-    if (c->batch <= 0 || c->n_pages <= 0 || c->max_pages <= 0) return CSA2_ERR_INVALID_ARG;
-    if ((int64_t)c->max_pages * CSA2_PAGE_ENTRIES > (int64_t)1 << 30) return CSA2_ERR_INVALID_ARG;
-    if (!aligned(c->pool, 256) || !aligned(c->swa, 256) || !aligned(c->pending, 16)) return CSA2_ERR_INVALID_ARG;
-    return CSA2_OK;
-}
-
 csa2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
 
 }  // namespace
@@ -91,6 +92,7 @@ csa2_status csa2_prefill(const csa2_cache *cache, int32_t req, int32_t m_host, i
                          int32_t n_tok_final, const float *lat, const float *key, const float *gate,
                          csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_prefill");
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
     if (req < 0 || req >= cache->batch || (m_host != 1 && m_host != 2)) return CSA2_ERR_INVALID_ARG;
@@ -107,6 +109,7 @@ csa2_status csa2_prefill(const csa2_cache *cache, int32_t req, int32_t m_host, i
 csa2_status csa2_append(const csa2_cache *cache, const float *lat, const float *key, const float *gate,
                         const int32_t *n_new, csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_append");
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
     if (!lat || !key || !gate || !n_new) return CSA2_ERR_INVALID_ARG;
@@ -118,6 +121,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
                        int32_t *pool, int32_t *pool_len, int32_t *topk, void *ws, size_t ws_bytes,
                        csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_index");
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
     if (!q_idx || !w || !topk || !ws || !aligned(ws, 256) || !aligned(q_idx, 16)) return CSA2_ERR_INVALID_ARG;
@@ -150,6 +154,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
 csa2_status csa2_topk(const float *scores, int64_t stride, const int32_t *n, int32_t batch, int32_t k,
                       int32_t *out, csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_topk");
     if (!scores || !n || !out || batch <= 0 || batch > 65535 || k < 1 || k > CSA2_MAX_BLOCKS || stride < 1)
         return CSA2_ERR_INVALID_ARG;
     if (stride > ((int64_t)1 << 31) / batch) return CSA2_ERR_INVALID_ARG;
@@ -164,6 +169,7 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
                         void *out, int32_t out_is_fp32, uint32_t flags, void *ws, size_t ws_bytes,
                         csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_attend");
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
     if (heads <= 0 || heads > 128 || !q || !topk || !out || !ws || !aligned(ws, 256)) return CSA2_ERR_INVALID_ARG;
@@ -181,6 +187,7 @@ csa2_status csa2_shard_blocks(const csa2_cache *shard, const int32_t *entry_offs
                               const float *w, int32_t *block_ids, float *block_scores, void *ws, size_t ws_bytes,
                               csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_shard_blocks");
     csa2_status st = check_cache(shard);
     if (st != CSA2_OK) return st;
     if (!entry_offset || !q_idx || !w || !block_ids || !block_scores || !ws || !aligned(ws, 256) ||
@@ -219,6 +226,7 @@ csa2_status csa2_shard_pool(const csa2_cache *shard, const int32_t *entry_offset
                             const int32_t *const *cand_ids, const float *const *cand_scores, int32_t *pool,
                             int32_t *pool_len, csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_shard_pool");
     csa2_status st = check_cache(shard);
     if (st != CSA2_OK) return st;
     ShardLists l;
@@ -232,6 +240,7 @@ csa2_status csa2_shard_rescore(const csa2_cache *shard, const int32_t *entry_off
                                const float *w, const int32_t *pool, const int32_t *pool_len, int32_t *ids,
                                float *scores, csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_shard_rescore");
     csa2_status st = check_cache(shard);
     if (st != CSA2_OK) return st;
     if (!entry_offset || !q_idx || !w || !pool || !pool_len || !ids || !scores || !aligned(q_idx, 16))
@@ -244,6 +253,7 @@ csa2_status csa2_shard_topk(const csa2_cache *shard, const int32_t *entry_offset
                             const int32_t *const *cand_ids, const float *const *cand_scores, int32_t *topk,
                             csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_shard_topk");
     csa2_status st = check_cache(shard);
     if (st != CSA2_OK) return st;
     ShardLists l;
@@ -257,6 +267,7 @@ csa2_status csa2_attend_partial(const csa2_cache *cache, int32_t heads, const ui
                                 float scale, int32_t with_window, float *o, float *lse, uint32_t flags,
                                 csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_attend_partial");
     csa2_status st = check_cache(cache);
     if (st != CSA2_OK) return st;
     if (heads <= 0 || heads > 128 || !q || !topk || !o || !lse) return CSA2_ERR_INVALID_ARG;
@@ -270,6 +281,7 @@ csa2_status csa2_attend_partial(const csa2_cache *cache, int32_t heads, const ui
 csa2_status csa2_combine(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts, int32_t batch,
                          int32_t heads, void *out, int32_t out_is_fp32, csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_combine");
     if (n_parts < 1 || n_parts > CSA2_MAX_SHARDS || !o_parts || !lse_parts || !out) return CSA2_ERR_INVALID_ARG;
     if (batch <= 0 || heads <= 0 || heads > 128 || (int64_t)batch * heads > 0x7fffffff || !aligned(out, 16))
         return CSA2_ERR_INVALID_ARG;
@@ -284,6 +296,7 @@ csa2_status csa2_combine(int32_t n_parts, const float *const *o_parts, const flo
 
 csa2_status csa2_get_device_error(const csa2_cache *cache, int32_t *code_out, csa2_stream_t stream)
 {
+    CSA2_TRACE("csa2_get_device_error");
     if (!cache || !cache->error || !code_out) return CSA2_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     int32_t v = 0;

@@ -7,11 +7,27 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <utility>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/csa2.h"
 
 namespace csa2 {
+
+// ---------------------------------------------------------------- tracing
+// An NVTX range around each C-ABI call, named after the call, so a profiler's
+// timeline shows which call enqueued which kernels (NVTX costs nothing when
+// no tool is attached).
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange &) = delete;
+    TraceRange &operator=(const TraceRange &) = delete;
+};
+#define CSA2_TRACE(name) ::csa2::TraceRange csa2_trace_range_(name)
 
 // ---------------------------------------------------------------- diagnostics
 // Defined in capi.cu: launch counting and optional event brackets.
@@ -22,6 +38,28 @@ struct LaunchScope {
     cudaStream_t st;
     LaunchScope(int kernel, cudaStream_t s) : k(kernel), st(s) { note_launch(k, st, true); }
     ~LaunchScope() { note_launch(k, st, false); }
+};
+
+// ---------------------------------------------------------------- one-time set-up
+// Per-device set-up of a launcher (function attributes, occupancy queries)
+// that host threads may reach concurrently: the first caller on a device runs
+// init under a lock; values init stores for that device are visible to every
+// caller that sees the flag set.
+struct DeviceOnce {
+    static constexpr int N = 64;
+    std::atomic<bool> done[N] = {};
+    std::mutex mu;
+    template <class F>
+    cudaError_t run(int dev, F &&init)
+    {
+        if (dev < 0 || dev >= N) return cudaErrorInvalidDevice;
+        if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lk(mu);
+        if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        const cudaError_t e = init();
+        if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+        return e;
+    }
 };
 
 // ---------------------------------------------------------------- launch order

@@ -134,28 +134,27 @@ cudaError_t launch_select(const CacheView &c, int src, const float *scores, int6
                           int32_t *pool_len, int max_n, cudaStream_t st, float *vals, const int32_t *id_off,
                           int id_shift)
 {
-    static bool attr_done[64] = {};
-    static int cluster_size[64] = {};
+    static DeviceOnce once;
+    static int cluster_size[DeviceOnce::N] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
     const int smem = (int)SEL_SMEM;
-    if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(select_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        const int nc = cluster_fits(select_cluster_kernel<16>, dim3(SEL_THREADS), smem, 16) ? 16 : 8;
-        if (dev < 64) {
-            cluster_size[dev] = nc;
-            attr_done[dev] = true;
-        }
-    }
-    const int nc = dev < 64 ? cluster_size[dev] : 8;
+    if (e == cudaSuccess)
+        e = once.run(dev, [&] {
+            cudaError_t r = cudaFuncSetAttribute(select_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (r == cudaSuccess)
+                cluster_size[dev] = cluster_fits(select_cluster_kernel<16>, dim3(SEL_THREADS), smem, 16) ? 16 : 8;
+            return r;
+        });
+    if (e != cudaSuccess) return e;
+    const int nc = cluster_size[dev];
     LaunchScope scope(CSA2_KERNEL_SELECT, st);
     if (max_n <= SEL_CAP)   // fits one CTA's shared memory: no cluster barriers on the path
         return launch_pdl(select_cta_kernel, dim3(1, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores, stride,

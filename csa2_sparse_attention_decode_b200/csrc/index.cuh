@@ -3,6 +3,11 @@
 #include "common.cuh"
 
 namespace csa2 {
+// Host-side validation of a cache descriptor shared by every entry point:
+// non-null fields, positive sizes, at most 2^30 entries per request, and
+// the pool / SWA ring 256-byte and pending 16-byte aligned.
+csa2_status check_cache(const csa2_cache *c);
+
 enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2, ROWS_GIVEN = 3 };
 
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,

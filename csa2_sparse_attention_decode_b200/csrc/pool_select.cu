@@ -318,27 +318,25 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
 {
     // 16 CTAs per request where the device can schedule such clusters
     // (shorter per-CTA row ranges), else 8.
-    static bool attr_done[64] = {};
-    static int cluster_size[64] = {};
+    static DeviceOnce once;
+    static int cluster_size[DeviceOnce::N] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = once.run(dev, [&] {
+            cudaError_t r = cudaFuncSetAttribute(pool_select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)Layout<8>::SMEM_BYTES);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Layout<16>::SMEM_BYTES);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (r == cudaSuccess)
+                cluster_size[dev] = cluster_fits(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16) ? 16 : 8;
+            return r;
+        });
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(pool_select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Layout<8>::SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)Layout<16>::SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        const int nc = cluster_fits(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16) ? 16 : 8;
-        if (dev < 64) {
-            cluster_size[dev] = nc;
-            attr_done[dev] = true;
-        }
-    }
-    const int nc = dev < 64 ? cluster_size[dev] : 8;
+    const int nc = cluster_size[dev];
     LaunchScope scope(CSA2_KERNEL_POOL_SCORE, st);
     if (nc == 16)
         return launch_pdl_cluster(pool_select_kernel<16>, dim3(16, c.batch), dim3(NT), Layout<16>::SMEM_BYTES, st, 16,

@@ -426,19 +426,6 @@ bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows)
     return r == CUDA_SUCCESS;
 }
 
-int sm_count()
-{
-    static int n[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (!n[dev]) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        n[dev] = v > 0 ? v : 148;
-    }
-    return n[dev];
-}
 
 }  // namespace
 
@@ -447,16 +434,21 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
 {
     (void)max_rows;
     if (c.batch > MAX_BATCH) return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
+    static DeviceOnce once;
+    static int n_sm[DeviceOnce::N] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = once.run(dev, [&] {
+            int v = 0;
+            cudaError_t r = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(score_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(SMEM_BYTES + 8 * (MAX_BATCH + 1)));
+            n_sm[dev] = v > 0 ? v : 148;
+            return r;
+        });
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(score_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(SMEM_BYTES + 8 * (MAX_BATCH + 1)));
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
-    }
     PlaneMaps maps;
     const long long np = c.n_pages;
     if (!make_plane_map(&maps.summ8, c.summ, np * 8, 8) || !make_plane_map(&maps.summ128, c.summ, np * 8, 128) ||
@@ -468,7 +460,7 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
                                                                                 : CSA2_KERNEL_POOL_SCORE;
     const size_t smem = SMEM_BYTES + 8 * ((size_t)c.batch + 1);
     LaunchScope scope(kid, st);
-    return launch_pdl(score_umma_kernel, dim3(CTAS_PER_SM * sm_count()), dim3(THREADS), smem, st, maps, p);
+    return launch_pdl(score_umma_kernel, dim3(CTAS_PER_SM * n_sm[dev]), dim3(THREADS), smem, st, maps, p);
 }
 
 }  // namespace csa2

@@ -197,15 +197,15 @@ __global__ void __launch_bounds__(128) combine_kernel(int n_parts, PartList p, i
 cudaError_t launch_shard_merge(const CacheView &c, const int32_t *entry_offset, int n_shards, const ShardLists &l,
                                int expand, int32_t *out, int32_t *pool_len, cudaStream_t st)
 {
-    static bool attr_done[64] = {};
+    static DeviceOnce once;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = once.run(dev, [] {
+            return cudaFuncSetAttribute(shard_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)MERGE_SMEM);
+        });
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev]) {
-        e = cudaFuncSetAttribute(shard_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MERGE_SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
-    }
     const int k = expand ? CSA2_MAX_BLOCKS : CSA2_TOPK;
     LaunchScope scope(CSA2_KERNEL_COMBINE, st);
     return launch_pdl(shard_merge_kernel, dim3(c.batch), dim3(MT), MERGE_SMEM, st, c, entry_offset, n_shards, l, k,

@@ -331,9 +331,14 @@ csa2_status csa2_combine(int32_t n_parts, const float *const *o_parts, const flo
  *     calls return CSA2_ERR_UNSUPPORTED and enqueue nothing.
  *   - The array (512 x 5 x 512 floats, about 5.2 MB) exists on every GPU
  *     that loads the library and stays allocated until the process exits.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.  No call allocates or frees memory.
+ *   - The first call on a device is set-up: with that device current it
+ *     looks up the array's device address (cudaGetSymbolAddress), and CUDA,
+ *     which loads a library's device code lazily by default, loads the
+ *     module that holds the array at that moment -- allocating the array's
+ *     device memory and possibly synchronising the device.  Make that first
+ *     call on each device while setting up, before any stream capture and
+ *     before the loop that must not allocate.  Later calls allocate and free
+ *     nothing.
  *   - All calls share the one array and each overwrites every partial it
  *     reads, so nothing carries over between calls; but two calls whose GPU
  *     work can overlap (different streams, or concurrent host threads
