@@ -106,7 +106,7 @@ def schedule_bytes(ws) -> dict:
 KNOWN_TRAFFIC = {
     "block_scan": {"bytes": 67_501_056 + 827_136, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
                    "sha256": "a3c2814836873bcbe6f19a489395cf2958005ce57066d43c01b840ceb548bc67"},
-    "attend": {"bytes": 1_557_504, "source": "csa2_sparse_attention_decode_b200/csrc/attend_dsm.cu",
+    "attend": {"bytes": 1_557_504, "source": "csa2_sparse_attention_decode_b200/csrc/attend.cu",
                "sha256": "cd3023c6207320cb71394114629a30235262131d546683ca4df14f43dd616b84"},
 }
 
@@ -230,7 +230,7 @@ def bench_config(w: synth.Workload) -> dict:
     return {"workload": w.name, "batch_per_gpu": w.batch, "entries_per_request": w.n_entries[0],
             "heads": w.heads, "layers": w.layers, "index": w.index,
             "l2": "flushed between timed steps (256 MB write, not timed)",
-            "timing": "CUDA graph replay of one step, CUDA events per step"}
+            "timing": "CUDA graph replay of one step (no event nodes inside), CUDA events around each replay"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) side
@@ -531,7 +531,7 @@ class Runner:
                 "caches": [{"name": c.name, "m": c.m[0], "layers": c.layers} for c in self.ws],
                 "kv_bytes_per_token": self.kv_bytes_per_token,
                 "l2": "flushed between timed steps (256 MB write, not timed)",
-                "timing": "CUDA graph replay of one step, CUDA events per step"}
+                "timing": "CUDA graph replay of one step (no event nodes inside), CUDA events around each replay"}
 
 
 def sharded_attend_bytes(rn) -> float:
@@ -601,34 +601,23 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     for p in rn.parts:
         assert csa2.csa2_get_device_error(p.cache, stream) == 0
 
-    # torch only reports elapsed time between events it has recorded itself;
-    # record each pair once so later records by the library are readable.
-    for ev in k_scan + k_att:
-        ev.record(stream)
-    stream.synchronize()
-    # One graph per layer: graph L brackets the attention of layer L (and the
-    # index scan) with events, so the timed replays, taken in turn, measure
-    # every layer's attention launch equally often.
-    scan_kernel = csa2.KERNEL_FLAT_SCORE if rn.flat else csa2.KERNEL_BLOCK_SCORE
-    csa2.csa2_set_profile_events(scan_kernel, *k_scan)
-    graphs = []
+    # The timed replays use a graph of the plain step: no event nodes inside,
+    # which would cut the programmatic-dependent-launch overlap between the
+    # kernels they separate.
+    step_graph = torch.cuda.CUDAGraph()
     n0 = csa2.csa2_launch_count()
-    for li in range(n_layers):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            rn.step(stream, attend_events=(li, k_att[0], k_att[1]))
-        graphs.append(g)
-    launches_per_step = (csa2.csa2_launch_count() - n0) / n_layers
-    csa2.csa2_set_profile_events(scan_kernel, None, None)
+    with torch.cuda.graph(step_graph, stream=stream):
+        rn.step(stream)
+    launches_per_step = csa2.csa2_launch_count() - n0
 
-    def one(i, timed_events=None):
+    def one(i, timed_events=None, graph=None):
         with torch.cuda.stream(stream):
             if rn.append:
                 rn.restore(stream)
             flush.zero_()
             if timed_events:
                 timed_events[0].record(stream)
-            graphs[i % n_layers].replay()
+            (graph or step_graph).replay()
             if timed_events:
                 timed_events[1].record(stream)
 
@@ -640,21 +629,56 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     sampler.mark(0)
-    step_ms, scan_ms, att_ms = [], [], []
+    step_ms = []
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
     for i in range(args.steps):
         e = ev[i % 2]
         one(i, e)
         stream.synchronize()
         step_ms.append(e[0].elapsed_time(e[1]))
-        scan_ms.append(k_scan[0].elapsed_time(k_scan[1]))
-        att_ms.append(k_att[0].elapsed_time(k_att[1]))
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     sampler.mark(1)
     max_total_ms = max_over_ranks(sum(step_ms), world, dev)
     value = job_throughput(world, rn.batch, args.steps, max_total_ms)
+
+    # ---- per-kernel device times, from separate replays of graphs whose
+    # chosen launches are bracketed by CUDA events recorded on the launching
+    # stream (graph L brackets layer L's attention, so taken in turn they
+    # cover every layer; the scan, block selection and pool kernels are
+    # bracketed in every graph, the pool pair keeping its last launch).
+    kern_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for k in ("scan", "select", "pool", "attend")}
+    for pair in kern_ev.values():          # torch reads elapsed times only of events it recorded once
+        for e_ in pair:
+            e_.record(stream)
+    stream.synchronize()
+    scan_kernel = csa2.KERNEL_FLAT_SCORE if rn.flat else csa2.KERNEL_BLOCK_SCORE
+    csa2.csa2_set_profile_events(scan_kernel, *kern_ev["scan"])
+    csa2.csa2_set_profile_events(csa2.KERNEL_SELECT, *kern_ev["select"])
+    csa2.csa2_set_profile_events(csa2.KERNEL_POOL_SCORE, *kern_ev["pool"])
+    diag = []
+    for li in range(n_layers):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            rn.step(stream, attend_events=(li, kern_ev["attend"][0], kern_ev["attend"][1]))
+        diag.append(g)
+    for k in (scan_kernel, csa2.KERNEL_SELECT, csa2.KERNEL_POOL_SCORE):
+        csa2.csa2_set_profile_events(k, None, None)
+    has_pool = any(m in ("full", "reindex") for w in rn.ws for m in w.layers) and not rn.flat
+    kt = {k: [] for k in kern_ev}
+    n_diag = max(n_layers, min(args.steps, 8 * n_layers))
+    for i in range(n_diag):
+        one(i, graph=diag[i % n_layers])
+        stream.synchronize()
+        for k, (e0, e1) in kern_ev.items():
+            if k == "pool" and not has_pool:
+                continue
+            kt[k].append(e0.elapsed_time(e1))
+    del diag
+    scan_ms, att_ms = kt["scan"], kt["attend"]
+    kernel_us = {k: 1000.0 * statistics.mean(v) for k, v in kt.items() if v}
 
     # ---- end to end: pinned host inputs -> device, replay, outputs -> host.
     # Pipelined as a serving loop runs it: one copy stream brings step i+1's
@@ -724,7 +748,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     att_avg_ms = statistics.mean(att_ms)
     att_bytes = ab["attend"] / n_layers if rn.sharded is None else sharded_attend_bytes(rn)
     att_gbs = att_bytes / (att_avg_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "attend_dsm_kernel", "achieved": att_gbs, "peak": peak,
+    roofline = {"bound": "hbm", "kernel": "attend_kernel", "achieved": att_gbs, "peak": peak,
                 "peak_source": peak_src, "unit": "GB/s", "frac": att_gbs / peak,
                 "traffic": known_traffic("attend"),
                 "kernel_ms": att_avg_ms, "launches_per_step": n_layers,
@@ -765,16 +789,21 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                                 "streams, overlapping the previous and next steps' compute; each step's device "
                                 "work (L2 flush, staging copies, the step) replayed as one CUDA graph"},
                 "gpu_launches": int(launches_per_step * args.steps),
+                "kernel_us": {"values": kernel_us,
+                              "how": "mean device time of one launch from separate replays with CUDA events "
+                                     "around it (scan = block or flat scan; select = block top-2048 or flat "
+                                     "top-512; pool = pool rescoring + top-512, the step's last; attend = "
+                                     "every layer in turn); the timed step graph holds no event nodes"},
                 "clocks": clocks}
         if per_shard is not None:
             # what each GPU of a G-GPU run would compute (its own shard's
             # kernels and the merges), without the exchanges between GPUs
             line["per_shard_ms_per_step"] = per_shard
-            roofline["kernel"] = "attend_dsm_kernel (the last shard's partial attention)"
+            roofline["kernel"] = "attend_kernel (the last shard's partial attention)"
             roofline_scan["kernel"] = "score_umma_kernel (the last shard's block-summary scan)"
             roofline["traffic"] = roofline_scan["traffic"] = None
         print(json.dumps(line), flush=True)
-    del graphs
+    del step_graph
     return line
 
 

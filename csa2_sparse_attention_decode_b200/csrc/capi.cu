@@ -50,7 +50,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 //   scores   [batch][row_stride] f32  row scores of the block or flat scan
 //   blocks   [batch][2048]       i32  selected blocks (FULL)
 // The pool's scores stay in shared memory (pool_select.cu) and attention
-// merges its splits inside a cluster (attend_dsm.cu): neither needs more.
+// merges its splits inside a cluster (attend.cu): neither needs more.
 struct Workspace {
     float *scores;
     int32_t *blocks;
@@ -178,8 +178,8 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
     Workspace W = layout(ws, cache->batch, heads, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
     if (flags & ~CSA2_ATTEND_INPUTS_SETTLED) return CSA2_ERR_INVALID_ARG;
-    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, flags, nullptr,
-                                   nullptr, (cudaStream_t)stream));
+    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, flags,
+                                   (cudaStream_t)stream));
 }
 
 // ------------------------------------------------------------ sequence shards
@@ -274,8 +274,7 @@ csa2_status csa2_attend_partial(const csa2_cache *cache, int32_t heads, const ui
     if (!aligned(o, 16) || !aligned(q, 16)) return CSA2_ERR_INVALID_ARG;
     if (flags & ~CSA2_ATTEND_INPUTS_SETTLED) return CSA2_ERR_INVALID_ARG;
     if (!with_window) flags |= ATT_NO_WINDOW;
-    return from_cuda(launch_attend_dsm(make_view(cache), heads, q, topk, scale, o, 1, flags, (cudaStream_t)stream,
-                                       lse));
+    return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, o, 1, flags, (cudaStream_t)stream, lse));
 }
 
 csa2_status csa2_combine(int32_t n_parts, const float *const *o_parts, const float *const *lse_parts, int32_t batch,

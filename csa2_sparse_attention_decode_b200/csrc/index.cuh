@@ -26,14 +26,12 @@ cudaError_t launch_prefill(const CacheView &c, int req, int m, int tok_begin, in
                            const float *lat, const float *key, const float *gate, cudaStream_t st);
 cudaError_t launch_append(const CacheView &c, const float *lat, const float *key, const float *gate,
                           const int32_t *n_new, cudaStream_t st);
-cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                          void *out, int out_is_fp32, uint32_t flags, float *part_o, float *part_ml, cudaStream_t st);
 
 // Attention with the split merge inside a cluster (distributed shared memory):
 // the csa2_attend path.  Needs no scratch.  With lse != nullptr it also
 // writes ln sum_j exp(scale * q.v_j) per (request, head) ([batch][heads]).
-cudaError_t launch_attend_dsm(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
-                              void *out, int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse = nullptr);
+cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
+                          void *out, int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse = nullptr);
 // Internal attention flag (beside CSA2_ATTEND_INPUTS_SETTLED): no window keys.
 constexpr uint32_t ATT_NO_WINDOW = 1u << 8;
 // Sequence-sharded decode (shard.cu): global top-k over the shards' lists,

@@ -9,9 +9,9 @@
 //
 // One cluster of NC = 16 CTAs per request (8 where 16 cannot be scheduled).
 // CTA r scores pool rows [r*chunk, r*chunk + chunk) (chunk a multiple of
-// 128, at most 16384 / NC) and keeps the
-// order-preserving keys of its scores in shared memory; the cluster then runs
-// the selection of select.cuh over them and writes the selected pool ids.
+// 128, at most 16384 / NC) and keeps the order-preserving keys of its scores
+// in shared memory; CTA 0 then gathers all of them and runs the selection of
+// select.cuh alone, writing the selected pool ids.
 // Scoring roles (384 threads):
 //   warps 5-11  look up the page of every 8-row run of the CTA's rows, then
 //               copy the runs (8 rows x 128 B of FP8 keys) with 16-byte
@@ -23,7 +23,7 @@
 //               four rotating accumulators;
 //   warps 0-3   split the query, then one thread per row: score =
 //               sum_h w'_h ReLU(D[h]);
-//   all warps then run the selection.
+//   then CTA 0's warps select.
 #include <cudaTypedefs.h>
 
 #include <cooperative_groups.h>
@@ -51,7 +51,7 @@ template <int NC>
 struct Layout {
     static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 2048 (NC = 8) or 1024 (NC = 16) rows
     static constexpr int RUNS = CHUNK_MAX / CSA2_BLOCK;  // runs of 8 rows
-    static constexpr int BITS_WORDS = CHUNK_MAX / 32;
+    static constexpr int BITS_WORDS = CSA2_POOL / 32;    // selection marks over the whole pool (CTA 0)
     static constexpr size_t OFF_Q = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t OFF_KEYS = OFF_Q + IQ_BYTES;
     static constexpr size_t OFF_CAND = OFF_KEYS + CHUNK_MAX * 4;
@@ -60,11 +60,13 @@ struct Layout {
     static constexpr size_t OFF_RUNS = OFF_BITS + BITS_WORDS * 4;
     static constexpr size_t SMEM_BYTES = 1024 + OFF_RUNS + RUNS * 4;
 };
-constexpr int ACC = 4;                                   // accumulators in tensor memory
-constexpr int ACC_COLS = CSA2_IDX_HEADS;                 // 32 columns each
-constexpr int QPART_BYTES = CSA2_IDX_HEADS * CSA2_KEY_DIM;
-constexpr uint32_t TMEM_COLS = ACC * ACC_COLS;           // 128
-// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, N = 32, M = 128.
+constexpr int ACC = 2;                                   // accumulators in tensor memory
+constexpr int ACC_COLS = IQ_ROWS;                        // 96 columns each: 3 query parts x 32 heads
+constexpr uint32_t TMEM_COLS = 256;                      // >= ACC * ACC_COLS, a power of two
+static_assert(ACC * ACC_COLS <= (int)TMEM_COLS, "tensor memory budget");
+// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, M = 128, N = 96:
+// the three query parts sit side by side as 96 B rows, so one MMA per
+// 32-dim K step scores a tile against all of them.
 constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(ACC_COLS >> 3) << 17) | (8u << 24);
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *err)
@@ -229,10 +231,8 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
                 const uint32_t aaddr = smem_addr(ring + s * STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < CSA2_KEY_DIM / 32; ++kk)
-#pragma unroll
-                    for (int pp = 0; pp < IQ_PARTS; ++pp)
-                        mma_f8(tb + ACC_COLS * ab, smem_desc(aaddr + kk * 32, 16, 1024),
-                               smem_desc(qaddr + pp * QPART_BYTES + kk * 32, 16, 1024), IDESC, (kk | pp) ? 1u : 0u);
+                    mma_f8(tb + ACC_COLS * ab, smem_desc(aaddr + kk * 32, 16, 1024),
+                           smem_desc(qaddr + kk * 32, 16, 1024), IDESC, kk > 0 ? 1u : 0u);
                 mma_commit(&d_full[ab]);
                 mma_commit(&empty[s]);                              // stage free once the MMAs have read it
             }
@@ -256,8 +256,10 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
             const int db = t % ACC;
             const bool ok = wait_or_abort(&d_full[db], (t / ACC) & 1, abort, c.error);
             fence_after_sync();
-            uint32_t r0[32];
+            uint32_t r0[32], r1[32], r2[32];                       // the three query parts' products
             tmem_ld32(tb + lane_base + ACC_COLS * db, r0);
+            tmem_ld32(tb + lane_base + ACC_COLS * db + 32, r1);
+            tmem_ld32(tb + lane_base + ACC_COLS * db + 64, r2);
             tmem_ld_wait();
             fence_before_sync();
             __syncwarp();
@@ -265,7 +267,10 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int hh = 0; hh < CSA2_IDX_HEADS; ++hh)
-                acc[hh & 3] = fmaf(wr[hh], fmaxf(__uint_as_float(r0[hh]), 0.0f), acc[hh & 3]);
+                acc[hh & 3] = fmaf(wr[hh],
+                                   fmaxf((__uint_as_float(r0[hh]) + __uint_as_float(r1[hh])) + __uint_as_float(r2[hh]),
+                                         0.0f),
+                                   acc[hh & 3]);
             const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             const int e = t * TILE + tid;
             if (e < cnt) {
@@ -278,10 +283,48 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     }
     fence_before_sync();
     __syncthreads();
+    if (warp == 5) {
+        fence_after_sync();
+        tmem_dealloc(tb, TMEM_COLS);
+    }
 
     // ---------------------------------------------------------------- selection
+    // CTA 0 gathers every CTA's keys (one round of 16-byte distributed-shared-
+    // memory loads, all in flight together) into its ring, now free, and
+    // selects alone: no cluster exchange inside the selection.
+    static_assert((size_t)STAGES * STAGE_BYTES >= (size_t)(CSA2_POOL + NT) * 4, "all keys fit the ring");
+    uint32_t *all = reinterpret_cast<uint32_t *>(ring);
+    cluster.sync();                                          // every CTA's keys final
+    kmin = 0xffffffffu;
+    kmax = 0u;
+    if (rank == 0) {
+        constexpr int G = 4;                                 // uint4 groups per thread per round
+        for (int g0 = 0; g0 < (n + 3) / 4; g0 += G * NT) {
+            uint4 v[G];
+#pragma unroll
+            for (int u = 0; u < G; ++u) {
+                const int g = g0 + u * NT + tid, e = 4 * g, r = e / max(chunk, 1);
+                v[u] = e < n ? reinterpret_cast<const uint4 *>(cluster.map_shared_rank(keys, r))[(e - r * chunk) >> 2]
+                             : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < G; ++u) {
+                const int e = 4 * (g0 + u * NT + tid);
+                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (e + j < n) {
+                        all[e + j] = w[j];
+                        kmin = min(kmin, w[j]);
+                        kmax = max(kmax, w[j]);
+                    }
+            }
+        }
+    }
+    cluster.sync();                                          // CTA 0 has read every CTA's keys
+    if (rank != 0) return;
     sel::Bufs bf;
-    bf.keys = keys;
+    bf.keys = all;
     bf.scores = nullptr;
     bf.cand_key = reinterpret_cast<uint32_t *>(sm + Lay::OFF_CAND);
     bf.cand_idx = bf.cand_key + sel::CAND;
@@ -300,14 +343,7 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     o.vals = topk_scores;
     o.id_off = id_off;
     o.id_shift = 0;
-    sel::select_core<NC, NT>(bf, b, n, chunk, lo, cnt, CSA2_TOPK, kmin, kmax, o);
-
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 5) {
-        fence_after_sync();
-        tmem_dealloc(tb, TMEM_COLS);
-    }
+    sel::select_core<1, NT>(bf, b, n, n, 0, n, CSA2_TOPK, kmin, kmax, o);
 }
 
 }  // namespace

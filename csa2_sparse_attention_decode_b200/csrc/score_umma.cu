@@ -39,14 +39,16 @@ constexpr int CTAS_PER_SM = 2;                              // two independent p
 constexpr int PW = 16;                                      // producer look-up window (tiles)
 constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;            // 16 KB
 constexpr int QBYTES = IQ_BYTES;                            // 3 parts x 32 heads x 128 dims of e5m2
-constexpr int QPART_BYTES = CSA2_IDX_HEADS * CSA2_KEY_DIM;  // 4 KB: one part
-constexpr int ACC = 4;                                      // accumulators in tensor memory
-constexpr int ACC_COLS = CSA2_IDX_HEADS;                    // 32 columns each
+constexpr int ACC = 2;                                      // accumulators in tensor memory
+constexpr int ACC_COLS = IQ_ROWS;                           // 96 columns each: 3 query parts x 32 heads
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = ACC * ACC_COLS;              // 128
+constexpr uint32_t TMEM_COLS = 256;                         // >= ACC * ACC_COLS, a power of two
+static_assert(ACC * ACC_COLS <= (int)TMEM_COLS && CTAS_PER_SM * TMEM_COLS <= 512, "tensor memory budget");
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + QBYTES;   // + 8 * (batch + 1)
 constexpr int MAX_BATCH = 1024;
-// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, N = 32, M = 128.
+// kind::f8f6f4: D f32, A e4m3 (0), B e5m2 (1), both K-major, M = 128, N = 96:
+// the three query parts sit side by side as 96 B rows, so one MMA per
+// 32-dim K step scores a tile against all of them.
 constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(ACC_COLS >> 3) << 17) | (8u << 24);
 
 // 2-D views (rows of 128 bytes) of the summary and key planes, with boxes of
@@ -351,10 +353,8 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
                 const uint32_t aaddr = smem_addr(sm + s * STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < CSA2_KEY_DIM / 32; ++kk)
-#pragma unroll
-                    for (int pp = 0; pp < IQ_PARTS; ++pp)
-                        mma_f8(tb + ACC_COLS * ab, smem_desc(aaddr + kk * 32, 16, 1024),
-                               smem_desc(qaddr + pp * QPART_BYTES + kk * 32, 16, 1024), IDESC, (kk | pp) ? 1u : 0u);
+                    mma_f8(tb + ACC_COLS * ab, smem_desc(aaddr + kk * 32, 16, 1024),
+                           smem_desc(qaddr + kk * 32, 16, 1024), IDESC, kk > 0 ? 1u : 0u);
                 mma_commit(&d_full[ab]);
                 mma_commit(&empty[s]);                              // stage free once the MMAs have read it
             }
@@ -387,8 +387,10 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             const int db = j % ACC;
             const bool ok = wait_or_abort(&d_full[db], (j / ACC) & 1, abort, p.c.error);
             fence_after_sync();
-            uint32_t r0[32];
+            uint32_t r0[32], r1[32], r2[32];                       // the three query parts' products
             tmem_ld32(tb + lane_base + ACC_COLS * db, r0);
+            tmem_ld32(tb + lane_base + ACC_COLS * db + 32, r1);
+            tmem_ld32(tb + lane_base + ACC_COLS * db + 64, r2);
             tmem_ld_wait();
             fence_before_sync();
             __syncwarp();
@@ -396,7 +398,10 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int hh = 0; hh < CSA2_IDX_HEADS; ++hh)
-                acc[hh & 3] = fmaf(wr[hh], fmaxf(__uint_as_float(r0[hh]), 0.0f), acc[hh & 3]);
+                acc[hh & 3] = fmaf(wr[hh],
+                                   fmaxf((__uint_as_float(r0[hh]) + __uint_as_float(r1[hh])) + __uint_as_float(r2[hh]),
+                                         0.0f),
+                                   acc[hh & 3]);
             const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             const int row = it.t * TILE + tid;
             if (ok && row < it.rows) p.scores[(size_t)it.b * p.stride + row] = sc;
