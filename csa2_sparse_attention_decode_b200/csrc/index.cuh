@@ -1,5 +1,7 @@
 // Launch entry points of the indexer kernels (host side).
 #pragma once
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 
 namespace csa2 {
@@ -9,6 +11,10 @@ namespace csa2 {
 csa2_status check_cache(const csa2_cache *c);
 
 enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2, ROWS_GIVEN = 3 };
+
+// 2-D TMA view of a 128-byte-row plane of the pool (keys or summaries):
+// `rows` rows, boxes of box_rows rows, 128-byte swizzled.  Host side.
+bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows);
 
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,
                          const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st);

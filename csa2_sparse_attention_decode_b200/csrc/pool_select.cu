@@ -9,13 +9,13 @@
 //
 // One cluster of NC = 16 CTAs per request (8 where 16 cannot be scheduled).
 // CTA r scores pool rows [r*chunk, r*chunk + chunk) (chunk a multiple of
-// 128, at most 16384 / NC) and keeps the order-preserving keys of its scores
-// in shared memory; CTA 0 then gathers all of them and runs the selection of
-// select.cuh alone, writing the selected pool ids.
+// 128, at most 16384 / NC) and keeps the
+// order-preserving keys of its scores in shared memory; the cluster then runs
+// the selection of select.cuh over them and writes the selected pool ids.
 // Scoring roles (384 threads):
-//   warps 5-11  look up the page of every 8-row run of the CTA's rows, then
-//               copy the runs (8 rows x 128 B of FP8 keys) with 16-byte
-//               asynchronous copies into an 8-stage ring of 128-row tiles,
+//   warps 5-11  look up the page of every 8-row run of the CTA's rows; warp
+//               5 then copies the runs (8 rows x 128 B of FP8 keys, 1 KB)
+//               with one TMA box each into an 8-stage ring of 128-row tiles,
 //               128-byte swizzled;
 //   warp 4      issues the MMAs: D[128 x 32] (fp32, tensor memory) =
 //               sum_p K[128 x 128] (e4m3) . Qp^T (kind::f8f6f4), Q1 + Q2 + Q3
@@ -23,7 +23,7 @@
 //               four rotating accumulators;
 //   warps 0-3   split the query, then one thread per row: score =
 //               sum_h w'_h ReLU(D[h]);
-//   then CTA 0's warps select.
+//   all warps then run the selection.
 #include <cudaTypedefs.h>
 
 #include <cooperative_groups.h>
@@ -51,7 +51,7 @@ template <int NC>
 struct Layout {
     static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 2048 (NC = 8) or 1024 (NC = 16) rows
     static constexpr int RUNS = CHUNK_MAX / CSA2_BLOCK;  // runs of 8 rows
-    static constexpr int BITS_WORDS = CSA2_POOL / 32;    // selection marks over the whole pool (CTA 0)
+    static constexpr int BITS_WORDS = CHUNK_MAX / 32;
     static constexpr size_t OFF_Q = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t OFF_KEYS = OFF_Q + IQ_BYTES;
     static constexpr size_t OFF_CAND = OFF_KEYS + CHUNK_MAX * 4;
@@ -91,21 +91,11 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
 __device__ __forceinline__ void bar_workers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void bar_producers() { asm volatile("bar.sync 2, %0;" ::"n"(NPROD) : "memory"); }
 
-// 16-byte asynchronous global -> shared copy (L2 only), and an arrival on an
-// mbarrier once every copy this thread issued before it has landed (the
-// arrival counts towards the barrier's expected count).
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 template <int NC>
-__global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const uint16_t *q_idx, const float *w, const int32_t *pool, const int32_t *pool_len,
-                   int32_t *topk, float *topk_scores, const int32_t *id_off)
+__global__ void __launch_bounds__(NT, 1)
+pool_select_kernel(const __grid_constant__ CUtensorMap map_keys8, CacheView c, const uint16_t *q_idx, const float *w,
+                   const int32_t *pool, const int32_t *pool_len, int32_t *topk, float *topk_scores,
+                   const int32_t *id_off)
 {
     using Lay = Layout<NC>;
     constexpr int RUNS = Lay::RUNS;
@@ -128,7 +118,7 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     }
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], NPROD);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < ACC; ++i) {
@@ -156,10 +146,9 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     if (warp >= 5 && n_tiles > 0) {
         // ------------------------------------------------------------ producers
         // Plane row of every run (pool id, then page table, each round's
-        // loads in flight together), then 16-byte asynchronous copies of the
-        // runs' rows into the ring, swizzled as the MMA reads them.  Gathered
-        // 1 KB runs are copied by the threads, not by TMA: a tile is 16 runs
-        // from unrelated pages.
+        // loads in flight together); then warp 5 copies each tile's 16 runs
+        // (8 rows x 128 B of one page, 1 KB) with one TMA box each, lanes
+        // 0-15 issuing together, 128-byte swizzled as the MMA reads them.
         const int ptid = tid - 5 * 32;
         const int n_runs = (cnt + CSA2_BLOCK - 1) / CSA2_BLOCK;
         constexpr int RPT = (RUNS + NPROD - 1) / NPROD;          // runs per producer thread
@@ -188,30 +177,28 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
             runs[j] = pid;
         }
         bar_producers();
-        int issued = 0;
-        for (int t = 0; t < n_tiles; ++t) {
-            const int s = t % STAGES;
-            bool okw = true;
-            if (lane == 0 && t >= STAGES) okw = wait_or_abort(&empty[s], ((t / STAGES) - 1) & 1, abort, c.error);
-            if (!__shfl_sync(0xffffffffu, okw, 0)) break;          // warp-uniform decision
-            uint8_t *stage = ring + s * STAGE_BYTES;
-            // 16 runs x 8 rows x 8 chunks of 16 bytes
-            for (int i = ptid; i < TILE * 8; i += NPROD) {
-                const int run = 16 * t + (i >> 6), r8 = (i >> 3) & 7, ch = i & 7;
-                const int pid = run < n_runs ? runs[run] : -1;
-                if (pid >= 0) {
-                    const int row = ((i >> 6) << 3) + r8;
-                    cp_async16(stage + row * 128 + ((ch ^ (row & 7)) << 4),
-                               c.keys + (size_t)(pid + r8) * CSA2_KEY_DIM + ch * 16);
-                }
+        if (warp == 5) {
+            if (lane == 0) tma_prefetch_map(&map_keys8);
+            int issued = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % STAGES;
+                bool okw = true;
+                if (lane == 0 && t >= STAGES) okw = wait_or_abort(&empty[s], ((t / STAGES) - 1) & 1, abort, c.error);
+                if (!__shfl_sync(0xffffffffu, okw, 0)) break;      // warp-uniform decision
+                uint8_t *stage = ring + s * STAGE_BYTES;
+                const int run = 16 * t + lane;
+                const int pid = (lane < 16 && run < n_runs) ? runs[run] : -1;
+                const uint32_t ok = __ballot_sync(0xffffffffu, pid >= 0);
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)__popc(ok) * CSA2_BLOCK * CSA2_KEY_DIM);
+                __syncwarp();
+                if (pid >= 0) tma_load_2d(stage + lane * CSA2_BLOCK * CSA2_KEY_DIM, &map_keys8, 0, pid, &full[s]);
+                issued = t + 1;
             }
-            cp_async_arrive(&full[s]);                              // one arrival per thread, when its copies land
-            issued = t + 1;
+            // Never leave with copies in flight: wait for the last stages to land.
+            if (lane == 0)
+                for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
+            __syncwarp();
         }
-        // Never leave with copies in flight: wait for the last stages to land.
-        if (lane == 0)
-            for (int j = max(0, issued - STAGES); j < issued; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1);
-        __syncwarp();
     } else if (warp == 4 && n_tiles > 0) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t qaddr = smem_addr(qbuf);
@@ -227,7 +214,6 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
             if (!__shfl_sync(0xffffffffu, okw, 0)) break;          // warp-uniform decision
             fence_after_sync();
             if (lane == 0) {
-                fence_proxy_async_smem();                           // the copies were generic-proxy writes
                 const uint32_t aaddr = smem_addr(ring + s * STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < CSA2_KEY_DIM / 32; ++kk)
@@ -283,48 +269,10 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
-        fence_after_sync();
-        tmem_dealloc(tb, TMEM_COLS);
-    }
 
     // ---------------------------------------------------------------- selection
-    // CTA 0 gathers every CTA's keys (one round of 16-byte distributed-shared-
-    // memory loads, all in flight together) into its ring, now free, and
-    // selects alone: no cluster exchange inside the selection.
-    static_assert((size_t)STAGES * STAGE_BYTES >= (size_t)(CSA2_POOL + NT) * 4, "all keys fit the ring");
-    uint32_t *all = reinterpret_cast<uint32_t *>(ring);
-    cluster.sync();                                          // every CTA's keys final
-    kmin = 0xffffffffu;
-    kmax = 0u;
-    if (rank == 0) {
-        constexpr int G = 4;                                 // uint4 groups per thread per round
-        for (int g0 = 0; g0 < (n + 3) / 4; g0 += G * NT) {
-            uint4 v[G];
-#pragma unroll
-            for (int u = 0; u < G; ++u) {
-                const int g = g0 + u * NT + tid, e = 4 * g, r = e / max(chunk, 1);
-                v[u] = e < n ? reinterpret_cast<const uint4 *>(cluster.map_shared_rank(keys, r))[(e - r * chunk) >> 2]
-                             : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < G; ++u) {
-                const int e = 4 * (g0 + u * NT + tid);
-                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (e + j < n) {
-                        all[e + j] = w[j];
-                        kmin = min(kmin, w[j]);
-                        kmax = max(kmax, w[j]);
-                    }
-            }
-        }
-    }
-    cluster.sync();                                          // CTA 0 has read every CTA's keys
-    if (rank != 0) return;
     sel::Bufs bf;
-    bf.keys = all;
+    bf.keys = keys;
     bf.scores = nullptr;
     bf.cand_key = reinterpret_cast<uint32_t *>(sm + Lay::OFF_CAND);
     bf.cand_idx = bf.cand_key + sel::CAND;
@@ -343,7 +291,14 @@ __global__ void __launch_bounds__(NT, 1) pool_select_kernel(CacheView c, const u
     o.vals = topk_scores;
     o.id_off = id_off;
     o.id_shift = 0;
-    sel::select_core<1, NT>(bf, b, n, n, 0, n, CSA2_TOPK, kmin, kmax, o);
+    sel::select_core<NC, NT>(bf, b, n, chunk, lo, cnt, CSA2_TOPK, kmin, kmax, o);
+
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        fence_after_sync();
+        tmem_dealloc(tb, TMEM_COLS);
+    }
 }
 
 }  // namespace
@@ -373,12 +328,15 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
         });
     if (e != cudaSuccess) return e;
     const int nc = cluster_size[dev];
+    CUtensorMap map_keys8;
+    if (!make_plane_map(&map_keys8, c.keys, (long long)c.n_pages * CSA2_PAGE_ENTRIES, CSA2_BLOCK))
+        return cudaErrorInvalidValue;
     LaunchScope scope(CSA2_KERNEL_POOL_SCORE, st);
     if (nc == 16)
         return launch_pdl_cluster(pool_select_kernel<16>, dim3(16, c.batch), dim3(NT), Layout<16>::SMEM_BYTES, st, 16,
-                                  c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
-    return launch_pdl_cluster(pool_select_kernel<8>, dim3(8, c.batch), dim3(NT), Layout<8>::SMEM_BYTES, st, 8, c,
-                              q_idx, w, pool, pool_len, topk, topk_scores, id_off);
+                                  map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
+    return launch_pdl_cluster(pool_select_kernel<8>, dim3(8, c.batch), dim3(NT), Layout<8>::SMEM_BYTES, st, 8,
+                              map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
 }
 
 }  // namespace csa2

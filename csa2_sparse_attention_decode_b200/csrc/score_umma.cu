@@ -415,6 +415,8 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
     }
 }
 
+}  // namespace
+
 // ---------------------------------------------------------------- host side
 // 2-D byte tensor over a plane: rows of 128 bytes, boxes of box_rows rows,
 // 128-byte swizzled.
@@ -430,9 +432,6 @@ bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows)
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
-
-
-}  // namespace
 
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,
                          const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st)

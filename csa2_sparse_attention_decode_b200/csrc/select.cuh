@@ -102,13 +102,14 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
                                             uint32_t kmin, uint32_t kmax, const Out &o)
 {
     constexpr int NW = NT / 32;
-    __shared__ uint32_t hist[2][256];
+    __shared__ __align__(16) uint32_t hist[2][256];
     __shared__ uint32_t whist[NW][256];
     __shared__ uint32_t scratch[32];
     __shared__ uint32_t wsum[NW][4];
-    __shared__ uint32_t s_cnt[4];
-    __shared__ uint32_t s_mm[4];
-    __shared__ uint32_t s_rk[NC][4];                       // per-rank values gathered by warp 0
+    __shared__ __align__(16) uint32_t s_cnt[4];
+    __shared__ __align__(16) uint32_t s_mm[4];
+    __shared__ __align__(16) uint32_t s_rk[NC][4];         // per-rank values gathered by warp 0
+    __shared__ uint32_t s_hsum[256];                       // cluster-wide histogram of a pass
 
     __shared__ uint32_t s_digit, s_above;
     const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
@@ -124,10 +125,18 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     // Warp 0 reads word(s) src[0..nw) of every CTA of the cluster into
     // s_rk[rank][..]; everyone else reads them from there (remote loads stay
     // NC * nw per CTA instead of per thread).
+    // One vector load per rank: src is 16-byte aligned (nw = 4), 8-byte
+    // aligned (nw = 2) or a single word.
     auto gather_ranks = [&](uint32_t *src, int nw) {
         if (wid == 0 && lane < NC) {
             const uint32_t *rc = remote(src, lane);
-            for (int i = 0; i < nw; ++i) s_rk[lane][i] = rc[i];
+            if (nw == 4) {
+                *reinterpret_cast<uint4 *>(&s_rk[lane][0]) = *reinterpret_cast<const uint4 *>(rc);
+            } else if (nw == 2) {
+                *reinterpret_cast<uint2 *>(&s_rk[lane][0]) = *reinterpret_cast<const uint2 *>(rc);
+            } else {
+                s_rk[lane][0] = rc[0];
+            }
         }
         __syncthreads();
     };
@@ -159,18 +168,18 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
             wsum[wid][3] = nthr;
         }
         __syncthreads();
-        if (tid == 0) {
-            uint32_t a = 0xffffffffu, z = 0u, l = 0xffffffffu, t = 0u;
-            for (int i = 0; i < NW; ++i) {
-                a = min(a, wsum[i][0]);
-                z = max(z, wsum[i][1]);
-                l = min(l, wsum[i][2]);
-                t += wsum[i][3];
+        if (wid == 0) {
+            const bool in = lane < NW;
+            const uint32_t a = __reduce_min_sync(0xffffffffu, in ? wsum[lane][0] : 0xffffffffu);
+            const uint32_t z = __reduce_max_sync(0xffffffffu, in ? wsum[lane][1] : 0u);
+            const uint32_t l = __reduce_min_sync(0xffffffffu, in ? wsum[lane][2] : 0xffffffffu);
+            const uint32_t t = __reduce_add_sync(0xffffffffu, in ? wsum[lane][3] : 0u);
+            if (lane == 0) {
+                s_mm[0] = a;
+                s_mm[1] = z;
+                s_mm[2] = l;
+                s_mm[3] = t;
             }
-            s_mm[0] = a;
-            s_mm[1] = z;
-            s_mm[2] = l;
-            s_mm[3] = t;
         }
         csync();
         gather_ranks(&s_mm[0], 4);
@@ -215,15 +224,24 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
             }
             __syncthreads();
             csync();
-            // Cluster-wide count of bin 255 - tid, then counts of bins >= it.
-            uint32_t hv = 0;
-            if (tid < 256) {
-                uint32_t part[NC];
+            // Cluster-wide counts: thread t < 64 sums bins 4t .. 4t + 3 over
+            // the CTAs with one 16-byte load each; then counts of bins >= b.
+            if (tid < 64) {
+                uint4 part[NC];
 #pragma unroll
-                for (int r = 0; r < NC; ++r) part[r] = remote(&hist[buf][0], r)[255 - tid];
+                for (int r = 0; r < NC; ++r) part[r] = reinterpret_cast<const uint4 *>(remote(&hist[buf][0], r))[tid];
+                uint4 a = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int r = 0; r < NC; ++r) hv += part[r];
+                for (int r = 0; r < NC; ++r) {
+                    a.x += part[r].x;
+                    a.y += part[r].y;
+                    a.z += part[r].z;
+                    a.w += part[r].w;
+                }
+                *reinterpret_cast<uint4 *>(&s_hsum[4 * tid]) = a;
             }
+            __syncthreads();
+            const uint32_t hv = tid < 256 ? s_hsum[255 - tid] : 0u;
             const uint32_t incl = scan256(hv, scratch);
             if (tid < 256 && incl >= krem && incl - hv < krem) {
                 s_digit = 255u - tid;
@@ -375,13 +393,16 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         }
         if (lane == 0) wsum[wid][1] = c;
         __syncthreads();
-        if (tid == 0) {
-            uint32_t a = 0;
-            for (int i = 0; i < NW; ++i) {
-                wsum[i][0] = a;
-                a += wsum[i][1];
+        if (wid == 0) {                                     // exclusive prefix over the warps
+            const uint32_t x = lane < NW ? wsum[lane][1] : 0u;
+            uint32_t y = x;
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const uint32_t t = __shfl_up_sync(0xffffffffu, y, o2);
+                if (lane >= o2) y += t;
             }
-            s_cnt[0] = a;
+            if (lane < NW) wsum[lane][0] = y - x;
+            if (lane == 31) s_cnt[0] = y;
         }
         __syncthreads();
         csync();
@@ -409,17 +430,26 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         wsum[wid][1] = neq;
     }
     __syncthreads();
-    if (tid == 0) {
-        uint32_t g = 0, q = 0;
-        for (int i = 0; i < NW; ++i) {
-            uint32_t a = wsum[i][0], bq = wsum[i][1];
-            wsum[i][0] = g;
-            wsum[i][1] = q;
-            g += a;
-            q += bq;
+    if (wid == 0) {                                         // exclusive prefixes over the warps
+        const uint32_t x0 = lane < NW ? wsum[lane][0] : 0u, x1 = lane < NW ? wsum[lane][1] : 0u;
+        uint32_t y0 = x0, y1 = x1;
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const uint32_t t0 = __shfl_up_sync(0xffffffffu, y0, o2), t1 = __shfl_up_sync(0xffffffffu, y1, o2);
+            if (lane >= o2) {
+                y0 += t0;
+                y1 += t1;
+            }
         }
-        s_cnt[0] = g;
-        s_cnt[1] = q;
+        __syncwarp();
+        if (lane < NW) {
+            wsum[lane][0] = y0 - x0;
+            wsum[lane][1] = y1 - x1;
+        }
+        if (lane == 31) {
+            s_cnt[0] = y0;
+            s_cnt[1] = y1;
+        }
     }
     __syncthreads();
     csync();
