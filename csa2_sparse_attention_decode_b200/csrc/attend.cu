@@ -17,7 +17,8 @@
 //   2. gather + dequantise 128 keys to bf16 (exact: e2m1 x e4m3 and
 //      e4m3 x 2^e all fit bf16) -> smem V tile, K-major, swizzled.  With
 //      CSA2_ATTEND_INPUTS_SETTLED this runs before the dependency wait.
-//   3. S^T[128 keys x HG heads] = V . Q^T             (32 MMAs, fp32 in TMEM)
+//   3. S^T[128 keys x HG heads] = V . Q^T  (32 MMAs from four issuers, one
+//      channel quarter and one fp32 TMEM accumulator each, summed on read)
 //   4. softmax per head over the tile's keys, in base 2: each warp takes the
 //      maximum of its 32 keys (TMEM lanes) with one warp reduction, the four
 //      lane groups meet in shared memory; P = 2^(x - m) is split into bf16
@@ -70,10 +71,12 @@ struct Cfg {
     // The staged output [head][dim] (fp32) reuses the V tile once the second
     // product has completed.
     static_assert(HG * CSA2_LATENT * 4 <= V_BYTES, "staging must fit the V tile");
-    // S^T in columns [0, HG); O^T chunk c in [2HG c, 2HG c + 2HG), written
-    // only after every S^T column has been read.
+    // S^T's four channel-quarter partials in columns [0, 4HG); O^T chunk c
+    // in [2HG c, 2HG c + 2HG), written only after every S^T column has been
+    // read.
     static constexpr uint32_t TMEM_COLS = 8 * HG;
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS >= 32, "allocation is a power of two");
+    static_assert(4 * HG <= (int)TMEM_COLS, "the S^T partials fit the allocation");
     static constexpr uint32_t IDESC_S = idesc_f16(128, HG, true, false, false);
     static constexpr uint32_t IDESC_O = idesc_f16(128, P_ROWS, true, true, false);
     static constexpr int TOTAL4 = HG * (CSA2_LATENT / 4);              // float4 of the output
@@ -292,7 +295,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
     const int nh = min(HG, heads - hg0);
     if (tid == 0) {
         mbar_init(&bar_q, 1);
-        mbar_init(&bar_s, 1);
+        mbar_init(&bar_s, 4);                                // one commit per issuing warp
         mbar_init(&bar_o, 4);                                // one commit per issuing warp
         mbar_fence_init();
         // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x HG heads, 128-byte
@@ -309,15 +312,18 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
     const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
 
     if (live) {
-        // ---- 3. S^T = V . Q^T
-        if (tid == 0) {
+        // ---- 3. S^T = V . Q^T, split along the 512 channels over four
+        // issuers (lane 0 of warps 0-3): issuer w sums channels [128w,
+        // 128w + 128) into its own accumulator, columns [HG w, HG w + HG).
+        if (lane == 0 && warp < 4) {
             wait_bar(&bar_q, 0, c.error);
             const uint32_t va = smem_addr(Vs), qa = smem_addr(Qs);
-#pragma unroll 4
-            for (int kk = 0; kk < CSA2_LATENT / 16; ++kk) {
+#pragma unroll
+            for (int j = 0; j < CSA2_LATENT / 64; ++j) {
+                const int kk = warp * (CSA2_LATENT / 64) + j;
                 const uint32_t off = (kk >> 2), in = (kk & 3) * 32;
-                mma_ss(tb, smem_desc(va + off * V_SLAB + in, 16, 1024), smem_desc(qa + off * Q_SLAB + in, 16, 1024),
-                       IDESC_S, kk > 0 ? 1u : 0u);
+                mma_ss(tb + (uint32_t)(HG * warp), smem_desc(va + off * V_SLAB + in, 16, 1024),
+                       smem_desc(qa + off * Q_SLAB + in, 16, 1024), IDESC_S, j > 0 ? 1u : 0u);
             }
             mma_commit(&bar_s);
         }
@@ -332,12 +338,19 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
     if (live) {
         float x[CPT];
         {
-            uint32_t rr[CPT];
-            ld_cols(tb + lane_base + c0, rr);
+            uint32_t r0[CPT], r1[CPT], r2[CPT], r3[CPT];        // the four channel quarters of S^T
+            ld_cols(tb + lane_base + c0, r0);
+            ld_cols(tb + lane_base + HG + c0, r1);
+            ld_cols(tb + lane_base + 2 * HG + c0, r2);
+            ld_cols(tb + lane_base + 3 * HG + c0, r3);
             tmem_ld_wait();
             const float sc2 = scale * LOG2E;
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) x[j] = valid ? __uint_as_float(rr[j]) * sc2 : -INFINITY;
+            for (int j = 0; j < CPT; ++j) {
+                const float sv = (__uint_as_float(r0[j]) + __uint_as_float(r1[j])) +
+                                 (__uint_as_float(r2[j]) + __uint_as_float(r3[j]));
+                x[j] = valid ? sv * sc2 : -INFINITY;
+            }
         }
         fence_before_sync();
 #pragma unroll

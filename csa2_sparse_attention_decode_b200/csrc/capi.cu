@@ -134,7 +134,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaSuccess;
     if (mode == CSA2_INDEX_FLAT) {
-        e = launch_score(c, ROWS_KEYS, q_idx, w, nullptr, nullptr, W.scores, W.row_stride, max_entries, s);
+        e = launch_score(c, ROWS_KEYS, q_idx, w, W.scores, W.row_stride, s);
         if (e == cudaSuccess)
             e = launch_select(c, ROWS_KEYS, W.scores, W.row_stride, nullptr, nullptr, CSA2_TOPK, topk, CSA2_TOPK,
                               0, nullptr, nullptr, max_entries, s);
@@ -142,7 +142,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
     }
     if (mode == CSA2_INDEX_FULL) {
         const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
-        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores, W.row_stride, max_blocks, s);
+        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, W.scores, W.row_stride, s);
         if (e == cudaSuccess)
             e = launch_select(c, ROWS_SUMMARIES, W.scores, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS,
                               W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, max_blocks, s);
@@ -199,7 +199,7 @@ csa2_status csa2_shard_blocks(const csa2_cache *shard, const int32_t *entry_offs
     CacheView c = make_view(shard);
     cudaStream_t s = (cudaStream_t)stream;
     const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
-    cudaError_t e = launch_score(c, ROWS_SUMMARIES, q_idx, w, nullptr, nullptr, W.scores, W.row_stride, max_blocks, s);
+    cudaError_t e = launch_score(c, ROWS_SUMMARIES, q_idx, w, W.scores, W.row_stride, s);
     if (e == cudaSuccess)
         e = launch_select(c, ROWS_SUMMARIES, W.scores, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS, block_ids,
                           CSA2_MAX_BLOCKS, 0, nullptr, nullptr, max_blocks, s, block_scores, entry_offset, 3);

@@ -68,6 +68,23 @@ struct DeviceOnce {
 // (completion and memory) before touching anything it may have written.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// A hint that brings the 128-byte line holding p into L2; it reads nothing
+// into the program, so it may run before griddepcontrol.wait: L2 is the
+// point of coherence, and the loads after the wait still see the producer's
+// writes.
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// Lanes of one warp hint the lines of bytes [lo, hi) of buf, at most
+// max_lines lines per lane.
+__device__ __forceinline__ void prefetch_l2_range(const void *buf, size_t lo, size_t hi, int lane, int max_lines)
+{
+    const char *b = static_cast<const char *>(buf);
+    lo &= ~(size_t)127;
+    for (int k = 0; k < max_lines; ++k) {
+        const size_t off = lo + ((size_t)k * 32 + lane) * 128;
+        if (off >= hi) break;
+        prefetch_l2(b + off);
+    }
+}
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,

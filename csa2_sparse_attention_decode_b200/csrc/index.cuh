@@ -16,8 +16,10 @@ enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2, ROWS_GIVEN = 
 // `rows` rows, boxes of box_rows rows, 128-byte swizzled.  Host side.
 bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows);
 
-cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,
-                         const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st);
+// Row scores of the block summaries (src ROWS_SUMMARIES) or of the keys
+// (ROWS_KEYS) of every request into scores[b * stride + row].
+cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, float *scores,
+                         int64_t stride, cudaStream_t st);
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
                           int32_t *pool_len, int max_n, cudaStream_t st, float *vals = nullptr,

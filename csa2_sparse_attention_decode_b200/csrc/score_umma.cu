@@ -51,10 +51,11 @@ constexpr int MAX_BATCH = 1024;
 // 32-dim K step scores a tile against all of them.
 constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(ACC_COLS >> 3) << 17) | (8u << 24);
 
-// 2-D views (rows of 128 bytes) of the summary and key planes, with boxes of
-// one 8-row run, one 64-row page and one whole 128-row tile.
+// 2-D views (rows of 128 bytes) of the summary plane (boxes of one page's
+// 8 rows and of a whole 128-row tile) and of the key plane (boxes of one
+// 64-row page and of a whole tile).
 struct PlaneMaps {
-    CUtensorMap summ8, summ128, keys8, keys64, keys128;
+    CUtensorMap summ8, summ128, keys64, keys128;
 };
 
 struct Params {
@@ -62,18 +63,14 @@ struct Params {
     int src;
     const uint16_t *q_idx;
     const float *w;
-    const int32_t *pool;
-    const int32_t *pool_len;
     float *scores;
     int64_t stride;
 };
 
 __device__ __forceinline__ int rows_of_req(const Params &p, int b)
 {
-    int n = n_entries_of(p.c, b);
-    if (p.src == ROWS_KEYS) return n;
-    if (p.src == ROWS_SUMMARIES) return (n + CSA2_BLOCK - 1) / CSA2_BLOCK;
-    return max(0, min(p.pool_len[b], CSA2_POOL));
+    const int n = n_entries_of(p.c, b);
+    return (p.src == ROWS_KEYS) ? n : (n + CSA2_BLOCK - 1) / CSA2_BLOCK;
 }
 
 // Walks this CTA's contiguous slice [i0, i1) of the global tile list, using
@@ -164,6 +161,19 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         mbar_fence_init();
     }
     int *s_rows = reinterpret_cast<int *>(qbuf + QBYTES), *s_pre = s_rows + p.c.batch;
+    if (warp == 4) {
+        // L2 hints while the previous kernel finishes: the request lengths,
+        // and this CTA's share of the page table and of the queries (all of
+        // them are hinted by the grid as a whole).
+        const size_t nb = (size_t)p.c.batch * 4;
+        prefetch_l2_range(p.c.n_tokens, 0, nb, lane, 8);
+        prefetch_l2_range(p.c.m, 0, nb, lane, 8);
+        const size_t pt = (size_t)p.c.batch * p.c.max_pages * 4, G = gridDim.x;
+        prefetch_l2_range(p.c.page_table, pt * blockIdx.x / G, pt * (blockIdx.x + 1) / G, lane, 16);
+        const size_t qb = (size_t)p.c.batch * CSA2_IDX_HEADS * CSA2_KEY_DIM * 2;
+        prefetch_l2_range(p.q_idx, qb * blockIdx.x / G, qb * (blockIdx.x + 1) / G, lane, 4);
+        if (blockIdx.x == 0) prefetch_l2_range(p.w, 0, (size_t)p.c.batch * CSA2_IDX_HEADS * 4, lane, 4);
+    }
     grid_dependency_wait();                      // inputs may come from the previous kernel
     allow_dependents();
     if (warp == 0) {
@@ -194,7 +204,12 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
     fence_after_sync();
     const uint32_t tb = tmem_base;
     const long long total = s_total;
-    const long long i0 = total * blockIdx.x / gridDim.x, i1 = total * (blockIdx.x + 1) / gridDim.x;
+    // [i0, i1) = [total * x / G, total * (x + 1) / G) with one 64-bit
+    // division: total = tq G + tr, tr < G, so the rest is 32-bit.
+    const uint32_t G = gridDim.x, x = blockIdx.x;
+    const long long tq = total / G;
+    const uint32_t tr = (uint32_t)(total - tq * G);
+    const long long i0 = tq * x + tr * x / G, i1 = tq * (x + 1) + tr * (x + 1) / G;
     const int n_items = (int)(i1 - i0);
     volatile int *abort = &s_abort;
 
@@ -206,8 +221,7 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         const int full_chunks = TILE / chunk_rows;                  // chunks of a complete tile
         const uint32_t chunk_bytes = (uint32_t)chunk_rows * CSA2_KEY_DIM;
         const int rows_per_page = (p.src == ROWS_SUMMARIES) ? 8 : 64;
-        const CUtensorMap *m_chunk = (p.src == ROWS_SUMMARIES) ? &maps.summ8 : (p.src == ROWS_KEYS) ? &maps.keys64
-                                                                                                  : &maps.keys8;
+        const CUtensorMap *m_chunk = (p.src == ROWS_SUMMARIES) ? &maps.summ8 : &maps.keys64;
         const CUtensorMap *m_tile = (p.src == ROWS_SUMMARIES) ? &maps.summ128 : &maps.keys128;
         if (lane == 0) {
             tma_prefetch_map(m_chunk);
@@ -219,7 +233,7 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         // Window w's look-ups go to buffer w & 1.  The page-table loads of
         // window w + 1 are issued before window w's copies and consumed after
         // them, so their latency hides behind the copies.
-        int e_[8], b_[8], pg_[8];
+        int e_[8], pg_[8];
         auto meta = [&](int w) {                    // lane i: tile i of window w
             const int wb = w & 1, nw = min(PW, n_items - w * PW);
             if (lane < nw) {
@@ -237,22 +251,20 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             __syncwarp();
         };
         auto issue_loads = [&](int w) {             // non-blocking: loads in flight
+            // Every lane loads for every u with no branch around the load (a
+            // load under a lane-divergent branch completes before the branch
+            // rejoins, which serialises the eight look-ups); a dead or
+            // out-of-range chunk reads entry 0, which always exists.
             const int wb = w & 1, nw = min(PW, n_items - w * PW);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int k = lane + 32 * u, i = k >> 4, ch = k & 15;
-                e_[u] = -1;
-                b_[u] = 0;
-                pg_[u] = -1;
-                if (i < nw && ch < win_n[wb][i]) {
-                    const int b = win_b[wb][i], r0 = win_r0[wb][i];
-                    b_[u] = b;
-                    if (p.src == ROWS_SUMMARIES) e_[u] = (r0 + 8 * ch) * CSA2_BLOCK;
-                    else if (p.src == ROWS_KEYS) e_[u] = r0 + 64 * ch;
-                    else e_[u] = p.pool[(size_t)b * CSA2_POOL + r0 + 8 * ch];
-                    if (p.src != ROWS_POOL && (e_[u] >> 6) < p.c.max_pages)
-                        pg_[u] = p.c.page_table[(size_t)b * p.c.max_pages + (e_[u] >> 6)];
-                }
+                const bool live = i < nw && ch < win_n[wb][i];
+                const int b = live ? win_b[wb][i] : 0, r0 = live ? win_r0[wb][i] : 0;
+                const int e = (p.src == ROWS_SUMMARIES) ? (r0 + 8 * ch) * CSA2_BLOCK : r0 + 64 * ch;
+                const bool in_pt = live && (e >> 6) < p.c.max_pages;
+                e_[u] = live ? e : -1;
+                pg_[u] = p.c.page_table[in_pt ? (size_t)b * p.c.max_pages + (e >> 6) : 0];
             }
         };
         auto finish = [&](int w) {                  // blocking: checks, then shared memory
@@ -260,29 +272,18 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int k = lane + 32 * u, i = k >> 4, ch = k & 15;
-                if (i >= nw) continue;
+                const int e = e_[u], pg = pg_[u];
                 int pid = -1;
-                if (ch < win_n[wb][i]) {
-                    int e = e_[u], pg = pg_[u];
-                    if (p.src == ROWS_POOL) {
-                        if (e < 0 || e >= n_entries_of(p.c, b_[u]) || (e & 7)) {
-                            set_error(p.c.error, CSA2_DEV_BAD_INDEX);
-                            e = -1;
-                        } else if ((e >> 6) < p.c.max_pages) {
-                            pg = p.c.page_table[(size_t)b_[u] * p.c.max_pages + (e >> 6)];
-                        }
-                    }
-                    if (e >= 0) {
-                        if ((e >> 6) >= p.c.max_pages) {
-                            set_error(p.c.error, CSA2_DEV_CAPACITY);
-                        } else if (pg < 0 || pg >= p.c.n_pages) {
-                            set_error(p.c.error, CSA2_DEV_BAD_PAGE);
-                        } else {
-                            pid = pg * rows_per_page + ((p.src == ROWS_SUMMARIES) ? 0 : (e & 63));   // plane row
-                        }
+                if (e >= 0) {
+                    if ((e >> 6) >= p.c.max_pages) {
+                        set_error(p.c.error, CSA2_DEV_CAPACITY);
+                    } else if (pg < 0 || pg >= p.c.n_pages) {
+                        set_error(p.c.error, CSA2_DEV_BAD_PAGE);
+                    } else {
+                        pid = pg * rows_per_page + ((p.src == ROWS_SUMMARIES) ? 0 : (e & 63));   // plane row
                     }
                 }
-                win_pid[wb][i][ch] = pid;
+                if (i < nw) win_pid[wb][i][ch] = pid;
             }
             __syncwarp();
         };
@@ -433,11 +434,10 @@ bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows)
     return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, const int32_t *pool,
-                         const int32_t *pool_len, float *scores, int64_t stride, int max_rows, cudaStream_t st)
+cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, float *scores,
+                         int64_t stride, cudaStream_t st)
 {
-    (void)max_rows;
-    if (c.batch > MAX_BATCH) return cudaErrorInvalidValue;
+    if (c.batch > MAX_BATCH || (src != ROWS_KEYS && src != ROWS_SUMMARIES)) return cudaErrorInvalidValue;
     static DeviceOnce once;
     static int n_sm[DeviceOnce::N] = {};
     int dev = 0;
@@ -456,12 +456,10 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
     PlaneMaps maps;
     const long long np = c.n_pages;
     if (!make_plane_map(&maps.summ8, c.summ, np * 8, 8) || !make_plane_map(&maps.summ128, c.summ, np * 8, 128) ||
-        !make_plane_map(&maps.keys8, c.keys, np * 64, 8) || !make_plane_map(&maps.keys64, c.keys, np * 64, 64) ||
-        !make_plane_map(&maps.keys128, c.keys, np * 64, 128))
+        !make_plane_map(&maps.keys64, c.keys, np * 64, 64) || !make_plane_map(&maps.keys128, c.keys, np * 64, 128))
         return cudaErrorInvalidValue;
-    Params p{c, src, q_idx, w, pool, pool_len, scores, stride};
-    int kid = src == ROWS_KEYS ? CSA2_KERNEL_FLAT_SCORE : src == ROWS_SUMMARIES ? CSA2_KERNEL_BLOCK_SCORE
-                                                                                : CSA2_KERNEL_POOL_SCORE;
+    Params p{c, src, q_idx, w, scores, stride};
+    const int kid = src == ROWS_KEYS ? CSA2_KERNEL_FLAT_SCORE : CSA2_KERNEL_BLOCK_SCORE;
     const size_t smem = SMEM_BYTES + 8 * ((size_t)c.batch + 1);
     LaunchScope scope(kid, st);
     return launch_pdl(score_umma_kernel, dim3(CTAS_PER_SM * n_sm[dev]), dim3(THREADS), smem, st, maps, p);

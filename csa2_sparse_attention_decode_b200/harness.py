@@ -75,10 +75,16 @@ class DeviceWorkload:
             self.cache.pending.copy_(self.saved_pending)
 
     # ------------------------------------------------------------ one step
-    def step(self, stream=None, attend_events=None):
+    def step(self, stream=None, attend_events=None, repeat=None):
         """One decode step.  attend_events = (layer, ev_start, ev_stop)
-        brackets that layer's attention launch with the two CUDA events."""
+        brackets that layer's attention launch with the two CUDA events.
+        repeat = {"attend" | "full" | "reindex": n} makes that call (every
+        attention, the Full layers' index, the Reindex layers' index) n
+        times in place; each repeat reads the same inputs and rewrites the
+        same outputs, so the step's results are unchanged and its extra time
+        is that call's cost inside the launch chain."""
         w, c = self.w, self.cache
+        rep = repeat or {}
         if w.append:
             lat, key, gate, n_new = self.new
             csa2_append(c, lat, key, gate, n_new, stream)
@@ -89,10 +95,13 @@ class DeviceWorkload:
             if mode == "full":
                 grp += 1
                 m = INDEX_FLAT if w.index == "flat" else INDEX_FULL
-                csa2_index(c, m, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws, stream)
+                for _ in range(rep.get("full", 1)):
+                    csa2_index(c, m, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws, stream)
             elif mode == "reindex":
                 grp += 1
-                csa2_index(c, INDEX_REINDEX, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws, stream)
+                for _ in range(rep.get("reindex", 1)):
+                    csa2_index(c, INDEX_REINDEX, q_idx, hw, self.pool, self.pool_len, self.topk[grp], self.ws,
+                               stream)
             buf = len(self.topk) - 1 if mode == "swa" else grp
             self.layer_topk.append(buf)
             # A Reuse layer's indices were produced by its group's first layer,
@@ -101,7 +110,8 @@ class DeviceWorkload:
             timed = attend_events is not None and attend_events[0] == li
             if timed:
                 csa2_set_profile_events(KERNEL_ATTEND, attend_events[1], attend_events[2])
-            csa2_attend(c, q, self.topk[buf], SOFTMAX_SCALE, self.outs[li], self.ws, stream, flags=flags)
+            for _ in range(rep.get("attend", 1)):
+                csa2_attend(c, q, self.topk[buf], SOFTMAX_SCALE, self.outs[li], self.ws, stream, flags=flags)
             if timed:
                 csa2_set_profile_events(KERNEL_ATTEND, None, None)
 
@@ -152,12 +162,13 @@ class ScheduleWorkload:
         for p in self.parts:
             p.restore(stream)
 
-    def step(self, stream=None, attend_events=None):
-        """attend_events = (global layer index, ev_start, ev_stop)."""
+    def step(self, stream=None, attend_events=None, repeat=None):
+        """attend_events = (global layer index, ev_start, ev_stop); repeat as
+        for DeviceWorkload.step."""
         base = 0
         for p in self.parts:
             ev = None
             if attend_events is not None and base <= attend_events[0] < base + len(p.w.layers):
                 ev = (attend_events[0] - base, attend_events[1], attend_events[2])
-            p.step(stream, attend_events=ev)
+            p.step(stream, attend_events=ev, repeat=repeat)
             base += len(p.w.layers)
