@@ -425,7 +425,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
     // memory loads: every tile's (m, l) into shared memory beside this
     // thread's five partial float4s, issued together.  Output (head h):
     //   out = sum_r 2^(m_r - M) O_r / sum_r l_r 2^(m_r - M),  M = max_r m_r.
-    cluster.sync();
+    cluster_sync_aligned();
     {
         const int lo4 = tile * TOTAL4 / NTILES, hi4 = (tile + 1) * TOTAL4 / NTILES;
         if (tid < 2 * NTILES * HG) {

@@ -68,6 +68,14 @@ struct DeviceOnce {
 // (completion and memory) before touching anything it may have written.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Cluster-wide barrier of every thread of every CTA of the cluster, in the
+// warp-aligned form (each warp arrives as one); every thread of each warp
+// must reach it together.  Release / acquire at cluster scope, as
+// cooperative_groups' cluster sync.
+__device__ __forceinline__ void cluster_sync_aligned()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // A hint that brings the 128-byte line holding p into L2; it reads nothing
 // into the program, so it may run before griddepcontrol.wait: L2 is the
 // point of coherence, and the loads after the wait still see the producer's

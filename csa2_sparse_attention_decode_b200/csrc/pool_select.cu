@@ -129,6 +129,20 @@ pool_select_kernel(const __grid_constant__ CUtensorMap map_keys8, CacheView c, c
         s_abort = 0;
         mbar_fence_init();
     }
+    if (warp == 6) {
+        // L2 hints while the previous kernel finishes (nothing is read before
+        // the wait): this CTA's share of request b's page table and of its
+        // indexer query, and the request's length.
+        const size_t pt = (size_t)c.max_pages * 4, qb = (size_t)CSA2_IDX_HEADS * CSA2_KEY_DIM * 2;
+        prefetch_l2_range(c.page_table + (size_t)b * c.max_pages, pt * rank / NC, pt * (rank + 1) / NC, lane, 16);
+        prefetch_l2_range(q_idx + (size_t)b * CSA2_IDX_HEADS * CSA2_KEY_DIM, qb * rank / NC, qb * (rank + 1) / NC,
+                          lane, 1);
+        if (rank == 0 && lane == 0) {
+            prefetch_l2(c.n_tokens + b);
+            prefetch_l2(c.m + b);
+            prefetch_l2(w + (size_t)b * CSA2_IDX_HEADS);
+        }
+    }
     grid_dependency_wait();                      // the pool may come from the previous kernel
     allow_dependents();
     const int n_entries = n_entries_of(c, b);
@@ -291,6 +305,9 @@ pool_select_kernel(const __grid_constant__ CUtensorMap map_keys8, CacheView c, c
     o.vals = topk_scores;
     o.id_off = id_off;
     o.id_shift = 0;
+    o.run_rows = runs;                           // the attention gathers the winners' latents next
+    o.codes = c.codes;
+    o.scales = c.scales;
     sel::select_core<NC, NT>(bf, b, n, chunk, lo, cnt, CSA2_TOPK, kmin, kmax, o);
 
     fence_before_sync();

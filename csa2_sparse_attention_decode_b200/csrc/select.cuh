@@ -65,6 +65,11 @@ struct Out {
     float *vals;                 // optional: the selected scores beside out (-inf padded)
     const int32_t *id_off;       // optional: (id_off[b] >> id_shift) is added to every written id
     int id_shift;
+    // Optional: the plane row of the first element of each local run of 8
+    // elements (shared memory, -1 if none).  Every selected element's latent
+    // code and scale lines are then hinted into L2 for the attention's gather.
+    const int32_t *run_rows = nullptr;
+    const uint8_t *codes = nullptr, *scales = nullptr;
 };
 
 // Inverse of ord_key (a -0 score comes back as +0).
@@ -114,7 +119,7 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     __shared__ uint32_t s_digit, s_above;
     const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
     auto csync = [&]() {
-        if constexpr (NC > 1) cg::this_cluster().sync();
+        if constexpr (NC > 1) cluster_sync_aligned();
         else __syncthreads();
     };
     auto remote = [&](uint32_t *ptr, int r) -> uint32_t * {
@@ -358,6 +363,15 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
             const int id = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
             o.out[(size_t)b * o.out_stride + pos] = (o.id_off && id >= 0) ? id + (o.id_off[b] >> o.id_shift) : id;
             if (o.vals) o.vals[(size_t)b * o.out_stride + pos] = key_score(key_at(gi - lo));
+            if (o.run_rows) {
+                const int li = gi - lo, r0 = o.run_rows[li >> 3];
+                if (r0 >= 0) {
+                    const size_t row = (size_t)r0 + (li & 7);
+                    prefetch_l2(o.codes + row * CSA2_CODE_BYTES);
+                    prefetch_l2(o.codes + row * CSA2_CODE_BYTES + 128);
+                    prefetch_l2(o.scales + row * CSA2_SCALE_BYTES);
+                }
+            }
         }
     };
     auto pad_tail = [&]() {
