@@ -56,12 +56,17 @@ constexpr int NTILES = ATT_SPLITS;          // 4 top-k tiles + the window = one 
 constexpr int V_SLAB = KT * 128;            // 16 KB: 128 keys x 64 dims (bf16)
 constexpr int V_BYTES = 8 * V_SLAB;         // 128 KB
 
-// Sizes for HG heads per CTA (16 or 32).
+// Sizes for HG heads per CTA (16, 24 or 32).
 template <int HG>
 struct Cfg {
-    static_assert(HG == 16 || HG == 32, "head group of 16 or 32");
+    static_assert(HG == 16 || HG == 24 || HG == 32, "head group of 16, 24 or 32");
     static constexpr int CPT = HG / 4;                 // softmax: S^T columns (heads) per thread
-    static constexpr int Q_SLAB = HG * 128;            // HG heads x 64 dims
+    static constexpr int CPT_LD = CPT == 6 ? 8 : CPT;  // columns loaded for them (a supported width)
+    // N of the first product: HG rounded up to a multiple of 16 (M = 128);
+    // q rows past HG in a slab are never written and their S^T columns never read.
+    static constexpr int SN = (HG + 15) / 16 * 16;
+    static constexpr int Q_SLAB = SN * 128;            // SN rows (HG heads) x 64 dims
+    static constexpr int Q_BOX_BYTES = 8 * HG * 128;   // what the eight q boxes bring
     static constexpr int Q_BYTES = 8 * Q_SLAB;
     static constexpr int P_ROWS = 2 * HG;              // hi rows, then lo rows
     static constexpr int P_SLAB = P_ROWS * 128;        // 2HG rows x 64 keys
@@ -71,13 +76,16 @@ struct Cfg {
     // The staged output [head][dim] (fp32) reuses the V tile once the second
     // product has completed.
     static_assert(HG * CSA2_LATENT * 4 <= V_BYTES, "staging must fit the V tile");
-    // S^T's four channel-quarter partials in columns [0, 4HG); O^T chunk c
-    // in [2HG c, 2HG c + 2HG), written only after every S^T column has been
-    // read.
-    static constexpr uint32_t TMEM_COLS = 8 * HG;
+    // S^T's four channel-quarter partials in columns [0, 4SN); O^T chunk c
+    // in [O_COL c, O_COL c + 2HG) (O_COL: 2HG rounded up to 32 columns),
+    // written only after every S^T column has been read.
+    static constexpr int O_COL = (2 * HG + 31) / 32 * 32;
+    static constexpr uint32_t TMEM_COLS = HG == 24 ? 256 : 8 * HG;
+    static_assert(4 * O_COL <= (int)TMEM_COLS, "the O^T chunks fit the allocation");
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS >= 32, "allocation is a power of two");
-    static_assert(4 * HG <= (int)TMEM_COLS, "the S^T partials fit the allocation");
-    static constexpr uint32_t IDESC_S = idesc_f16(128, HG, true, false, false);
+    static_assert(4 * SN <= (int)TMEM_COLS && 8 * HG <= (int)TMEM_COLS, "the accumulators fit the allocation");
+    static_assert(3 * CPT + CPT_LD <= SN, "softmax loads stay inside one S^T partial");
+    static constexpr uint32_t IDESC_S = idesc_f16(128, SN, true, false, false);
     static constexpr uint32_t IDESC_O = idesc_f16(128, P_ROWS, true, true, false);
     static constexpr int TOTAL4 = HG * (CSA2_LATENT / 4);              // float4 of the output
     static constexpr int NU = (TOTAL4 / NTILES + 1 + THREADS - 1) / THREADS;   // per thread in the merge
@@ -124,7 +132,8 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
     return *reinterpret_cast<uint32_t *>(&r);
 }
 
-// Tensor-memory load of as many columns as the array holds.
+// Tensor-memory load of as many columns as the array holds (4, 8, 16, 32,
+// 48 or 64).
 template <int N>
 __device__ __forceinline__ void ld_cols(uint32_t a, uint32_t (&r)[N])
 {
@@ -136,6 +145,11 @@ __device__ __forceinline__ void ld_cols(uint32_t a, uint32_t (&r)[N])
         tmem_ld16(a, r);
     } else if constexpr (N == 32) {
         tmem_ld32(a, r);
+    } else if constexpr (N == 48) {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[0]);
+        uint32_t (&hi)[16] = *reinterpret_cast<uint32_t (*)[16]>(&r[32]);
+        tmem_ld32(a, lo);
+        tmem_ld16(a + 32, hi);
     } else {
         static_assert(N == 64, "4 to 64 columns");
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[0]);
@@ -300,7 +314,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
         mbar_fence_init();
         // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x HG heads, 128-byte
         // swizzled (K-major operand layout); heads past `heads` read as zero.
-        mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
+        mbar_arrive_expect_tx(&bar_q, C::Q_BOX_BYTES);
         for (int slab = 0; slab < 8; ++slab) tma_load_3d(Qs + slab * Q_SLAB, &map_q, 64 * slab, hg0, b, &bar_q);
     }
     if (!early) gather();
@@ -314,7 +328,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
     if (live) {
         // ---- 3. S^T = V . Q^T, split along the 512 channels over four
         // issuers (lane 0 of warps 0-3): issuer w sums channels [128w,
-        // 128w + 128) into its own accumulator, columns [HG w, HG w + HG).
+        // 128w + 128) into its own accumulator, columns [SN w, SN w + SN).
         if (lane == 0 && warp < 4) {
             wait_bar(&bar_q, 0, c.error);
             const uint32_t va = smem_addr(Vs), qa = smem_addr(Qs);
@@ -322,7 +336,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
             for (int j = 0; j < CSA2_LATENT / 64; ++j) {
                 const int kk = warp * (CSA2_LATENT / 64) + j;
                 const uint32_t off = (kk >> 2), in = (kk & 3) * 32;
-                mma_ss(tb + (uint32_t)(HG * warp), smem_desc(va + off * V_SLAB + in, 16, 1024),
+                mma_ss(tb + (uint32_t)(C::SN * warp), smem_desc(va + off * V_SLAB + in, 16, 1024),
                        smem_desc(qa + off * Q_SLAB + in, 16, 1024), IDESC_S, j > 0 ? 1u : 0u);
             }
             mma_commit(&bar_s);
@@ -338,11 +352,11 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
     if (live) {
         float x[CPT];
         {
-            uint32_t r0[CPT], r1[CPT], r2[CPT], r3[CPT];        // the four channel quarters of S^T
+            uint32_t r0[C::CPT_LD], r1[C::CPT_LD], r2[C::CPT_LD], r3[C::CPT_LD];   // the four channel quarters
             ld_cols(tb + lane_base + c0, r0);
-            ld_cols(tb + lane_base + HG + c0, r1);
-            ld_cols(tb + lane_base + 2 * HG + c0, r2);
-            ld_cols(tb + lane_base + 3 * HG + c0, r3);
+            ld_cols(tb + lane_base + C::SN + c0, r1);
+            ld_cols(tb + lane_base + 2 * C::SN + c0, r2);
+            ld_cols(tb + lane_base + 3 * C::SN + c0, r3);
             tmem_ld_wait();
             const float sc2 = scale * LOG2E;
 #pragma unroll
@@ -388,7 +402,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
             for (int kk = 0; kk < KT / 16; ++kk) {
                 const uint64_t ad = smem_desc(va + (2 * cc) * V_SLAB + kk * 2048, V_SLAB, 1024);
                 const uint64_t bd = smem_desc(pa + (kk >> 2) * P_SLAB + (kk & 3) * 32, 16, 1024);
-                mma_ss(tb + (uint32_t)(2 * HG * cc), ad, bd, IDESC_O, kk > 0 ? 1u : 0u);
+                mma_ss(tb + (uint32_t)(C::O_COL * cc), ad, bd, IDESC_O, kk > 0 ? 1u : 0u);
             }
             mma_commit(&bar_o);
         }
@@ -409,7 +423,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
         fence_after_sync();
         const int cc = warp >> 2;
         uint32_t rr[2 * HG];
-        ld_cols(tb + lane_base + (uint32_t)(2 * HG * cc), rr);
+        ld_cols(tb + lane_base + (uint32_t)(C::O_COL * cc), rr);
         tmem_ld_wait();
         const int d = 128 * cc + 32 * sp + lane;
 #pragma unroll
@@ -530,15 +544,19 @@ cudaError_t launch_hg(const CacheView &c, int heads, const uint16_t *q, const in
 
 }  // namespace
 
-// 16-head CTAs halve each CTA's softmax, staging and merge work (the
-// latency of a small batch) but gather every key twice as often; they are
-// used while all their clusters run on the device at once (one wave),
-// 32-head CTAs beyond that.  A request with at most 16 heads takes 16.
+// Head groups: 16-head CTAs halve each CTA's softmax, staging and merge work
+// (the latency of a small batch) but gather every key more often.  16 heads
+// while all of a launch's clusters run at once (one wave), 24 while those
+// do, 32 beyond.  (Fewer, larger CTAs would let consecutive launches be
+// resident together, but at a batch of 4 x 64 heads 24-head CTAs measured
+// 10.2 us per launch in a chain against 10.0 for 16-head ones: their merge
+// costs more than the residency saves.)  A request with at most 16 heads
+// takes 16.
 cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, const int32_t *topk, float scale,
                           void *out, int out_is_fp32, uint32_t flags, cudaStream_t st, float *lse)
 {
     static DeviceOnce once;
-    static int wave16[DeviceOnce::N] = {};
+    static int wave16[DeviceOnce::N] = {}, wave24[DeviceOnce::N] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
@@ -546,32 +564,47 @@ cudaError_t launch_attend(const CacheView &c, int heads, const uint16_t *q, cons
             cudaError_t r = cudaFuncSetAttribute(attend_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)Cfg<16>::SMEM_BYTES);
             if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(attend_kernel<24>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<24>::SMEM_BYTES);
+            if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(attend_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg<32>::SMEM_BYTES);
             if (r != cudaSuccess) return r;
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(NTILES, 1, 1);
-            cfg.blockDim = dim3(THREADS, 1, 1);
-            cfg.dynamicSmemBytes = Cfg<16>::SMEM_BYTES;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = NTILES;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, (void *)attend_kernel<16>, &cfg) != cudaSuccess) {
-                cudaGetLastError();
-                n = 0;
-            }
-            wave16[dev] = n;
+            auto clusters = [&](const void *fn, size_t smem) {
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3(NTILES, 1, 1);
+                cfg.blockDim = dim3(THREADS, 1, 1);
+                cfg.dynamicSmemBytes = smem;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = NTILES;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+                    cudaGetLastError();
+                    n = 0;
+                }
+                return n;
+            };
+            wave16[dev] = clusters((const void *)attend_kernel<16>, Cfg<16>::SMEM_BYTES);
+            wave24[dev] = clusters((const void *)attend_kernel<24>, Cfg<24>::SMEM_BYTES);
             return cudaSuccess;
         });
     if (e != cudaSuccess) return e;
     const long long clusters16 = (long long)((heads + 15) / 16) * c.batch;
+    const long long clusters24 = (long long)((heads + 23) / 24) * c.batch;
+    int hg;
     if (heads <= 16 || clusters16 <= wave16[dev])
-        return launch_hg<16>(c, heads, q, topk, scale, out, out_is_fp32, flags, st, lse);
+        hg = 16;
+    else if (clusters24 <= wave24[dev])
+        hg = 24;
+    else
+        hg = 32;
+    if (hg == 16) return launch_hg<16>(c, heads, q, topk, scale, out, out_is_fp32, flags, st, lse);
+    if (hg == 24) return launch_hg<24>(c, heads, q, topk, scale, out, out_is_fp32, flags, st, lse);
     return launch_hg<32>(c, heads, q, topk, scale, out, out_is_fp32, flags, st, lse);
 }
 
