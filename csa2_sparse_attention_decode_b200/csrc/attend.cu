@@ -303,24 +303,36 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
                     *reinterpret_cast<uint4 *>(vrow + s * V_SLAB + (ch << 4)) = make_uint4(0, 0, 0, 0);
         }
     };
-    if (early) gather();                                  // inputs settled: overlap the previous kernel
-    grid_dependency_wait();                               // q (and, unless settled, the rest) may be fresh
-    allow_dependents();
-    const int nh = min(HG, heads - hg0);
     if (tid == 0) {
         mbar_init(&bar_q, 1);
         mbar_init(&bar_s, 4);                                // one commit per issuing warp
         mbar_init(&bar_o, 4);                                // one commit per issuing warp
         mbar_fence_init();
+    }
+    // Settled inputs: the gather, and the CTA barrier that publishes it (and
+    // the tensor-memory base and the mbarriers), overlap the previous kernel.
+    bool live = false;                                    // any valid key in this tile
+    if (early) {
+        gather();
+        fence_proxy_async_smem();
+        live = __syncthreads_or(valid) != 0;
+        fence_after_sync();
+    }
+    grid_dependency_wait();                               // q (and, unless settled, the rest) may be fresh
+    allow_dependents();
+    const int nh = min(HG, heads - hg0);
+    if (tid == 0) {
         // ---- 1. q -> smem by TMA: 8 boxes of 64 dims x HG heads, 128-byte
         // swizzled (K-major operand layout); heads past `heads` read as zero.
         mbar_arrive_expect_tx(&bar_q, C::Q_BOX_BYTES);
         for (int slab = 0; slab < 8; ++slab) tma_load_3d(Qs + slab * Q_SLAB, &map_q, 64 * slab, hg0, b, &bar_q);
     }
-    if (!early) gather();
-    fence_proxy_async_smem();
-    const bool live = __syncthreads_or(valid) != 0;      // any valid key in this tile
-    fence_after_sync();
+    if (!early) {
+        gather();
+        fence_proxy_async_smem();
+        live = __syncthreads_or(valid) != 0;
+        fence_after_sync();
+    }
     const uint32_t tb = tmem_base;
     const int sp = warp & 3;                              // TMEM lane group: keys / dims 32 sp ..
     const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
