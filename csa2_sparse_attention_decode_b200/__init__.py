@@ -64,7 +64,7 @@ def _load():
     sig = {
         "csa2_page_bytes": (SZ, []),
         "csa2_swa_bytes": (SZ, []),
-        "csa2_workspace_bytes": (SZ, [I32, I32, I32]),
+        "csa2_workspace_bytes": (SZ, [I32, I32]),
         "csa2_prefill": (C.c_int, [P, I32, I32, I32, I32, I32, P, P, P, P]),
         "csa2_append": (C.c_int, [P, P, P, P, P, P]),
         "csa2_index": (C.c_int, [P, C.c_int, P, P, P, P, P, P, SZ, P]),
@@ -161,12 +161,12 @@ def csa2_swa_bytes() -> int:
     return int(lib.csa2_swa_bytes())
 
 
-def csa2_workspace_bytes(batch: int, heads: int, max_entries: int) -> int:
-    return int(lib.csa2_workspace_bytes(batch, heads, max_entries))
+def csa2_workspace_bytes(batch: int, max_entries: int) -> int:
+    return int(lib.csa2_workspace_bytes(batch, max_entries))
 
 
-def workspace(cache: Cache, heads: int) -> torch.Tensor:
-    n = csa2_workspace_bytes(cache.batch, heads, cache.max_entries)
+def workspace(cache: Cache) -> torch.Tensor:
+    n = csa2_workspace_bytes(cache.batch, cache.max_entries)
     return torch.empty(n, dtype=torch.uint8, device=cache.device)
 
 

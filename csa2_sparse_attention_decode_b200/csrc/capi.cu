@@ -58,13 +58,12 @@ struct Workspace {
     size_t bytes;
 };
 
-Workspace layout(void *base, int32_t batch, int32_t heads, int32_t max_entries)
+Workspace layout(void *base, int32_t batch, int32_t max_entries)
 {
     Workspace w{};
     w.row_stride = ((int64_t)max_entries + 3) & ~(int64_t)3;
     size_t off = 0;
     auto take = [&](size_t n) { size_t o = off; off = align256(off + n); return (char *)base + o; };
-    (void)heads;
     w.scores = (float *)take(sizeof(float) * (size_t)batch * (size_t)w.row_stride);
     w.blocks = (int32_t *)take(sizeof(int32_t) * (size_t)batch * CSA2_MAX_BLOCKS);
     w.bytes = off;
@@ -82,10 +81,10 @@ extern "C" {
 size_t csa2_page_bytes(void) { return CSA2_PAGE_BYTES; }
 size_t csa2_swa_bytes(void) { return CSA2_SWA_BYTES; }
 
-size_t csa2_workspace_bytes(int32_t batch, int32_t heads, int32_t max_entries)
+size_t csa2_workspace_bytes(int32_t batch, int32_t max_entries)
 {
-    if (batch <= 0 || heads <= 0 || max_entries < 0) return 0;
-    return layout(nullptr, batch, heads, max_entries).bytes;
+    if (batch <= 0 || max_entries < 0) return 0;
+    return layout(nullptr, batch, max_entries).bytes;
 }
 
 csa2_status csa2_prefill(const csa2_cache *cache, int32_t req, int32_t m_host, int32_t tok_begin, int32_t n_tok,
@@ -128,7 +127,7 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
     if (mode != CSA2_INDEX_FLAT && mode != CSA2_INDEX_FULL && mode != CSA2_INDEX_REINDEX) return CSA2_ERR_INVALID_ARG;
     if (mode != CSA2_INDEX_FLAT && (!pool || !pool_len)) return CSA2_ERR_INVALID_ARG;
     const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
-    Workspace W = layout(ws, cache->batch, 1, max_entries);
+    Workspace W = layout(ws, cache->batch, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
     CacheView c = make_view(cache);
     cudaStream_t s = (cudaStream_t)stream;
@@ -175,7 +174,7 @@ csa2_status csa2_attend(const csa2_cache *cache, int32_t heads, const uint16_t *
     if (heads <= 0 || heads > 128 || !q || !topk || !out || !ws || !aligned(ws, 256)) return CSA2_ERR_INVALID_ARG;
     if (!aligned(out, 16) || !aligned(q, 16)) return CSA2_ERR_INVALID_ARG;
     const int max_entries = cache->max_pages * CSA2_PAGE_ENTRIES;
-    Workspace W = layout(ws, cache->batch, heads, max_entries);
+    Workspace W = layout(ws, cache->batch, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
     if (flags & ~CSA2_ATTEND_INPUTS_SETTLED) return CSA2_ERR_INVALID_ARG;
     return from_cuda(launch_attend(make_view(cache), heads, q, topk, scale, out, out_is_fp32, flags,
@@ -194,7 +193,7 @@ csa2_status csa2_shard_blocks(const csa2_cache *shard, const int32_t *entry_offs
         !aligned(q_idx, 16))
         return CSA2_ERR_INVALID_ARG;
     const int max_entries = shard->max_pages * CSA2_PAGE_ENTRIES;
-    Workspace W = layout(ws, shard->batch, 1, max_entries);
+    Workspace W = layout(ws, shard->batch, max_entries);
     if (ws_bytes < W.bytes) return CSA2_ERR_INVALID_ARG;
     CacheView c = make_view(shard);
     cudaStream_t s = (cudaStream_t)stream;

@@ -38,7 +38,7 @@ class DeviceWorkload:
         for li in range(len(w.layers)):
             q, q_idx, hw = synth.queries(w, li)
             self.layers.append((q.to(self.device), q_idx.to(self.device), hw.to(self.device)))
-        self.ws = workspace(self.cache, w.heads)
+        self.ws = workspace(self.cache)
         B = w.batch
         self.pool = torch.full((B, POOL), -1, dtype=torch.int32, device=self.device)
         self.pool_len = torch.zeros(B, dtype=torch.int32, device=self.device)

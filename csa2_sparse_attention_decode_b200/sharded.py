@@ -108,7 +108,7 @@ class Shard:
         self.cache, self.heads, self.last = cache, heads, last
         dev, B = cache.device, cache.batch
         self.entry_offset = torch.tensor(list(offsets), dtype=torch.int32, device=dev)
-        self.ws = workspace(cache, heads)
+        self.ws = workspace(cache)
         self.blk_ids = torch.full((B, MAX_BLOCKS), -1, dtype=torch.int32, device=dev)
         self.blk_scores = torch.full((B, MAX_BLOCKS), float("-inf"), dtype=torch.float32, device=dev)
         self.pool = torch.full((B, POOL), -1, dtype=torch.int32, device=dev)
