@@ -290,12 +290,14 @@ def test_empty_request_and_partial_head_group():
     check_attention(dw.outs[0][0], r, "request 0, 40 heads")
 
 
-def test_partial_head_group_in_both_cta_shapes():
-    """40 heads in a batch small enough for 16-head attention CTAs (2
-    requests) and in one too large for a single wave of them (40 requests,
-    32-head CTAs: one full group and a partial one); sampled requests of
-    both against the oracle."""
-    for batch, picks in ((2, (0, 1)), (40, (0, 17, 39))):
+def test_partial_head_group_in_every_cta_shape():
+    """40 heads in a batch small enough for one wave of 16-head attention
+    CTAs (2 requests), in one whose 16-head clusters exceed a wave but whose
+    24-head ones do not (12 requests on a 148-SM part: a full 24-head group
+    and a partial one of 16), and in one too large for both (40 requests,
+    32-head CTAs: one full group and a partial one); sampled requests of each
+    against the oracle, whichever CTA shape the launch picks."""
+    for batch, picks in ((2, (0, 1)), (12, (0, 5, 11)), (40, (0, 17, 39))):
         w = synth.Workload(f"heads40-B{batch}", 9, batch, 40, [2500] * batch, [1] * batch, "flat", ["full"], False)
         dw = DeviceWorkload(w, out_fp32=True)
         dw.step()
@@ -311,10 +313,15 @@ def test_partial_head_group_in_both_cta_shapes():
             check_attention(dw.outs[0][b], ref.attend(bits(q[b]), top, SOFTMAX_SCALE), f"B={batch} request {b}")
 
 
-def test_maximum_heads():
-    """128 query heads, the most csa2_attend takes (eight 16-head groups per
-    request), with Full and Reuse layers, against the oracle."""
-    w = synth.Workload("heads128-B2", 13, 2, 128, [6000, 3001], [1, 2], "hier", ["full", "reuse"], False)
+@pytest.mark.parametrize("batch", [2, 4])
+def test_maximum_heads(batch):
+    """128 query heads, the most csa2_attend takes, with Full and Reuse
+    layers, against the oracle: 2 requests (eight 16-head groups each) and 4
+    (on a 148-SM part, 24-head CTAs: five full groups and a partial one of 8
+    heads)."""
+    n_tok = [6000, 3001, 4500, 2000][:batch]
+    w = synth.Workload(f"heads128-B{batch}", 13, batch, 128, n_tok, [1, 2, 1, 2][:batch], "hier",
+                       ["full", "reuse"], False)
     dw = DeviceWorkload(w, out_fp32=True)
     refs = [OracleRequest(w, b, w.n_tok[b]) for b in range(w.batch)]
     check_step(w, dw, refs)
