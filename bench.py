@@ -106,8 +106,8 @@ def schedule_bytes(ws) -> dict:
 KNOWN_TRAFFIC = {
     "block_scan": {"bytes": 67_488_256 + 385_280, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
                    "sha256": "af7d26568d8ef087acaec3d0c826b96c248ba4328756b62ba52cd6683641f923"},
-    "attend": {"bytes": 1_552_640, "source": "csa2_sparse_attention_decode_b200/csrc/attend.cu",
-               "sha256": "e438955b17b17cd5ebd42127ae6793990485ff44d4e0f685c027cefe68ada343"},
+    "attend": {"bytes": 1_553_280, "source": "csa2_sparse_attention_decode_b200/csrc/attend.cu",
+               "sha256": "40e39a5ebdbad81ec1002ccbbc3b4bf478252c2806a42203d6616b70aca74982"},
 }
 
 
