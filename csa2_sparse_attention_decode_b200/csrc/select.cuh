@@ -113,8 +113,9 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     __shared__ uint32_t wsum[NW][4];
     __shared__ __align__(16) uint32_t s_cnt[4];
     __shared__ __align__(16) uint32_t s_mm[4];
-    __shared__ __align__(16) uint32_t s_rk[NC][4];         // per-rank values gathered by warp 0
+    __shared__ __align__(16) uint32_t s_rk[NC][4];         // per-rank candidate counts, gathered by warp 0
     __shared__ uint32_t s_hsum[256];                       // cluster-wide histogram of a pass
+    __shared__ uint32_t s_g[4];                            // cluster-wide reductions, formed by warp 0
 
     __shared__ uint32_t s_digit, s_above;
     const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
@@ -127,24 +128,6 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         else return ptr;
     };
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    // Warp 0 reads word(s) src[0..nw) of every CTA of the cluster into
-    // s_rk[rank][..]; everyone else reads them from there (remote loads stay
-    // NC * nw per CTA instead of per thread).
-    // One vector load per rank: src is 16-byte aligned (nw = 4), 8-byte
-    // aligned (nw = 2) or a single word.
-    auto gather_ranks = [&](uint32_t *src, int nw) {
-        if (wid == 0 && lane < NC) {
-            const uint32_t *rc = remote(src, lane);
-            if (nw == 4) {
-                *reinterpret_cast<uint4 *>(&s_rk[lane][0]) = *reinterpret_cast<const uint4 *>(rc);
-            } else if (nw == 2) {
-                *reinterpret_cast<uint2 *>(&s_rk[lane][0]) = *reinterpret_cast<const uint2 *>(rc);
-            } else {
-                s_rk[lane][0] = rc[0];
-            }
-        }
-        __syncthreads();
-    };
     const int kk = min(k, n);
     const bool take_all = n <= k;
     const int seg = ((cnt + NW * 32 - 1) / (NW * 32)) * 32;     // elements per warp, multiple of 32
@@ -187,14 +170,20 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
             }
         }
         csync();
-        gather_ranks(&s_mm[0], 4);
-        uint32_t gmin = 0xffffffffu, gmax = 0u, glb = 0xffffffffu, gthr = 0u;
-        for (int r = 0; r < NC; ++r) {
-            gmin = min(gmin, s_rk[r][0]);
-            gmax = max(gmax, s_rk[r][1]);
-            glb = min(glb, s_rk[r][2]);
-            gthr += s_rk[r][3];
+        if (wid == 0) {                                     // one 16-byte load per rank, reduced in the warp
+            uint4 v = make_uint4(0xffffffffu, 0u, 0xffffffffu, 0u);
+            if (lane < NC) v = *reinterpret_cast<const uint4 *>(remote(&s_mm[0], lane));
+            const uint32_t a = __reduce_min_sync(0xffffffffu, v.x), z = __reduce_max_sync(0xffffffffu, v.y);
+            const uint32_t l = __reduce_min_sync(0xffffffffu, v.z), t = __reduce_add_sync(0xffffffffu, v.w);
+            if (lane == 0) {
+                s_g[0] = a;
+                s_g[1] = z;
+                s_g[2] = l;
+                s_g[3] = t;
+            }
         }
+        __syncthreads();
+        const uint32_t gmin = s_g[0], gmax = s_g[1], glb = s_g[2], gthr = s_g[3];
         const uint32_t low = gthr >= (uint32_t)kk ? glb : gmin;
         int hi = 32 - __clz(low ^ gmax);                    // bits [hi-1 .. 0] vary above `low`
         pmask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
@@ -284,14 +273,17 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
                 static_assert(NC * (CAND + 1) < (1 << 30) && CAND + 1 > RANK_MAX, "candidate count encoding");
                 if (tid == 0) s_cnt[3] = use_cand ? (uint32_t)n_cand : (uint32_t)(CAND + 1);
                 csync();
-                __syncthreads();                            // s_rk is reused
-                gather_ranks(&s_cnt[3], 1);
-                uint32_t total = 0, most = 0;
-                for (int r = 0; r < NC; ++r) {
-                    const uint32_t v = s_rk[r][0];
-                    total += v;
-                    most = max(most, v);
+                if (wid == 0) {                             // every rank's count, their sum and maximum
+                    const uint32_t v = lane < NC ? *remote(&s_cnt[3], lane) : 0u;
+                    const uint32_t tot = __reduce_add_sync(0xffffffffu, v), mo = __reduce_max_sync(0xffffffffu, v);
+                    if (lane < NC) s_rk[lane][0] = v;
+                    if (lane == 0) {
+                        s_g[0] = tot;
+                        s_g[1] = mo;
+                    }
                 }
+                __syncthreads();
+                const uint32_t total = s_g[0], most = s_g[1];
                 // Rank directly when the comparisons per lane stay small (the
                 // same decision in every CTA of the cluster).
                 const uint32_t work = ((most + NW - 1) / NW) * ((total + 31) / 32);
@@ -420,9 +412,13 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         }
         __syncthreads();
         csync();
-        gather_ranks(&s_cnt[0], 1);
-        uint32_t base = wsum[wid][0];
-        for (int r = 0; r < rank; ++r) base += s_rk[r][0];
+        if (wid == 0) {                                     // the counts of the lower ranks, summed
+            const uint32_t v = lane < rank ? *remote(&s_cnt[0], lane) : 0u;
+            const uint32_t pre = __reduce_add_sync(0xffffffffu, v);
+            if (lane == 0) s_g[0] = pre;
+        }
+        __syncthreads();
+        const uint32_t base = wsum[wid][0] + s_g[0];
         // Nobody reads this CTA's shared memory after this point.
         if constexpr (NC > 1) asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
         const uint32_t nw = wsum[wid][1];
@@ -467,14 +463,17 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     }
     __syncthreads();
     csync();
-    gather_ranks(&s_cnt[0], 2);
-    uint32_t gt_b = 0, eq_b = 0;
-    for (int r = 0; r < rank; ++r) {
-        gt_b += s_rk[r][0];
-        eq_b += s_rk[r][1];
+    if (wid == 0) {                                         // the lower ranks' counts, summed
+        uint2 v = make_uint2(0u, 0u);
+        if (lane < rank) v = *reinterpret_cast<const uint2 *>(remote(&s_cnt[0], lane));
+        const uint32_t p0 = __reduce_add_sync(0xffffffffu, v.x), p1 = __reduce_add_sync(0xffffffffu, v.y);
+        if (lane == 0) {
+            s_g[0] = p0;
+            s_g[1] = p1;
+        }
     }
-    gt_b += wsum[wid][0];
-    eq_b += wsum[wid][1];
+    __syncthreads();
+    uint32_t gt_b = s_g[0] + wsum[wid][0], eq_b = s_g[1] + wsum[wid][1];
     for (int it = 0; it < seg; it += 32) {
         const int e = wid * seg + it + lane;
         const bool valid = e < cnt;
