@@ -108,7 +108,7 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
 {
     constexpr int NW = NT / 32;
     __shared__ __align__(16) uint32_t hist[2][256];
-    __shared__ uint32_t whist[NW][256];
+    __shared__ __align__(16) uint32_t whist[NW][256];
     __shared__ uint32_t scratch[32];
     __shared__ uint32_t wsum[NW][4];
     __shared__ __align__(16) uint32_t s_cnt[4];
@@ -193,7 +193,7 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         for (int pass = 0; hi > 0; ++pass) {
             const int wdt = min(8, hi), shift = hi - wdt, buf = pass & 1;
             const uint32_t dmask = (1u << wdt) - 1u;
-            for (int i = tid; i < NW * 256; i += NT) whist[i >> 8][i & 255] = 0;
+            for (int i = tid; i < NW * 64; i += NT) reinterpret_cast<uint4 *>(&whist[0][0])[i] = make_uint4(0, 0, 0, 0);
             __syncthreads();
             if (use_cand) {
                 for (int ci = tid; ci < n_cand; ci += NT) {
@@ -347,9 +347,15 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     const uint32_t lt_mask = (1u << lane) - 1u;
     auto write_one = [&](int gi, uint32_t pos) {
         if (o.expand) {
-            for (int j = 0; j < CSA2_BLOCK; ++j) {
-                const int en = gi * CSA2_BLOCK + j;
-                o.pool[(size_t)b * CSA2_POOL + pos * CSA2_BLOCK + j] = en < o.n_entries ? en : -1;
+            static_assert(CSA2_BLOCK == 8, "a block's entries are two int4");
+            int32_t *dst = o.pool + (size_t)b * CSA2_POOL + (size_t)pos * CSA2_BLOCK;
+            const int e0 = gi * CSA2_BLOCK, ne = o.n_entries;
+            auto id = [&](int j) { return e0 + j < ne ? e0 + j : -1; };
+            if ((reinterpret_cast<uintptr_t>(o.pool) & 15) == 0) {     // two 16-byte stores per block
+                reinterpret_cast<int4 *>(dst)[0] = make_int4(id(0), id(1), id(2), id(3));
+                reinterpret_cast<int4 *>(dst)[1] = make_int4(id(4), id(5), id(6), id(7));
+            } else {
+                for (int j = 0; j < CSA2_BLOCK; ++j) dst[j] = id(j);
             }
         } else {
             const int id = o.ids ? o.ids[(size_t)b * CSA2_POOL + gi] : gi;
@@ -384,7 +390,11 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         // elements in place (over keys it has already read), then the
         // warps' and CTAs' counts place them.  (Not with scores out: the
         // compaction overwrites the keys.)
+        // (The pool length, known to the thread holding the last element, is
+        // stored after the cluster barriers: a global store before one would
+        // hold up its release.)
         uint32_t c = 0;
+        int pool_len_out = -1;
         for (int it = 0; it < seg; it += 32) {
             const int e = wid * seg + it + lane;
             const bool valid = e < cnt;
@@ -395,7 +405,7 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
             if (chosen) bf.keys[wid * seg + c + __popc(bal & lt_mask)] = (uint32_t)e;
             c += __popc(bal);
             if (o.expand && valid && lo + e == n - 1)
-                o.pool_len[b] = kk * CSA2_BLOCK - (chosen ? n * CSA2_BLOCK - o.n_entries : 0);
+                pool_len_out = kk * CSA2_BLOCK - (chosen ? n * CSA2_BLOCK - o.n_entries : 0);
         }
         if (lane == 0) wsum[wid][1] = c;
         __syncthreads();
@@ -423,6 +433,7 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
         if constexpr (NC > 1) asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
         const uint32_t nw = wsum[wid][1];
         for (uint32_t j = lane; j < nw; j += 32) write_one(lo + (int)bf.keys[wid * seg + j], base + j);
+        if (pool_len_out >= 0) o.pool_len[b] = pool_len_out;
         pad_tail();
         if constexpr (NC > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
         return;
@@ -474,6 +485,10 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     }
     __syncthreads();
     uint32_t gt_b = s_g[0] + wsum[wid][0], eq_b = s_g[1] + wsum[wid][1];
+    // Nobody reads another CTA's shared memory after this point: arrive now,
+    // wait only after the output stores (a release after them would wait
+    // for them).
+    if constexpr (NC > 1) asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
     for (int it = 0; it < seg; it += 32) {
         const int e = wid * seg + it + lane;
         const bool valid = e < cnt;
@@ -491,7 +506,8 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     }
     pad_tail();
     // No CTA may leave while another still reads its shared memory.
-    csync();
+    if constexpr (NC > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    else __syncthreads();
 }
 
 }  // namespace sel
