@@ -251,10 +251,12 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             __syncwarp();
         };
         auto issue_loads = [&](int w) {             // non-blocking: loads in flight
-            // Every lane loads for every u with no branch around the load (a
-            // load under a lane-divergent branch completes before the branch
-            // rejoins, which serialises the eight look-ups); a dead or
-            // out-of-range chunk reads entry 0, which always exists.
+            // Every lane loads for every u with no branch around the load: with
+            // each load under a lane-divergent branch the eight look-ups of a
+            // lane were measured to complete one after another (eight memory
+            // latencies); unconditional loads from clamped addresses are in
+            // flight together.  A dead or out-of-range chunk reads entry 0,
+            // which always exists.
             const int wb = w & 1, nw = min(PW, n_items - w * PW);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
