@@ -49,8 +49,7 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     const int n_entries = (src == ROWS_GIVEN) ? 0 : n_entries_of(c, b);
     const int n = (src == ROWS_KEYS) ? n_entries
                 : (src == ROWS_SUMMARIES) ? (n_entries + CSA2_BLOCK - 1) / CSA2_BLOCK
-                : (src == ROWS_POOL) ? max(0, min(pool_len_in[b], CSA2_POOL))
-                                     : (int)max((int64_t)0, min((int64_t)pool_len_in[b], score_stride));
+                                          : (int)max((int64_t)0, min((int64_t)pool_len_in[b], score_stride));
     const int chunk = (n + NC - 1) / NC;
     const int lo = rank * chunk;
     const int cnt = max(0, min(n, lo + chunk) - lo);

@@ -10,7 +10,9 @@ namespace csa2 {
 // the pool / SWA ring 256-byte and pending 16-byte aligned.
 csa2_status check_cache(const csa2_cache *c);
 
-enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_POOL = 2, ROWS_GIVEN = 3 };
+// What a scan or a selection runs over: every key of the requests, their
+// block summaries, or (selection only) a given score matrix with row lengths.
+enum RowSource { ROWS_KEYS = 0, ROWS_SUMMARIES = 1, ROWS_GIVEN = 2 };
 
 // 2-D TMA view of a 128-byte-row plane of the pool (keys or summaries):
 // `rows` rows, boxes of box_rows rows, 128-byte swizzled.  Host side.
