@@ -200,8 +200,8 @@ __device__ __forceinline__ uint32_t kmajor_off(int n, int k, int slab_bytes)
 
 template <int HG>
 __global__ void __cluster_dims__(NTILES, 1, 1) __launch_bounds__(THREADS, 1)
-attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads, const int32_t *topk, float scale,
-              void *out, int out_is_fp32, uint32_t flags, float *lse)
+attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads, const int32_t *topk, const uint16_t *q,
+              float scale, void *out, int out_is_fp32, uint32_t flags, float *lse)
 {
     using C = Cfg<HG>;
     constexpr int CPT = C::CPT, Q_SLAB = C::Q_SLAB, P_SLAB = C::P_SLAB, NU = C::NU;
@@ -226,6 +226,12 @@ attend_kernel(const __grid_constant__ CUtensorMap map_q, CacheView c, int heads,
         fence_before_sync();
     }
     if (tid == 32) tma_prefetch_map(&map_q);
+    if (warp == 1) {
+        // An L2 hint of this tile's fifth of the group's q rows (nothing is
+        // read before the wait; the copy after it sees the current data).
+        const size_t row0 = (size_t)b * heads + hg0, nb = (size_t)min(HG, heads - hg0) * CSA2_LATENT * 2;
+        prefetch_l2_range(q + row0 * CSA2_LATENT, nb * tile / NTILES, nb * (tile + 1) / NTILES, lane, 2);
+    }
     const bool early = (flags & CSA2_ATTEND_INPUTS_SETTLED) != 0;
     bool valid = false;
     // ---- 2. key `row`, channels [128*qtr, 128*qtr + 128) -> slabs 2*qtr, 2*qtr + 1
@@ -550,7 +556,7 @@ cudaError_t launch_hg(const CacheView &c, int heads, const uint16_t *q, const in
     if (!make_q_map(&map_q, q, heads, c.batch, HG)) return cudaErrorInvalidValue;
     dim3 grid(NTILES, (heads + HG - 1) / HG, c.batch);
     LaunchScope scope(CSA2_KERNEL_ATTEND, st);
-    return launch_pdl(attend_kernel<HG>, grid, dim3(THREADS), Cfg<HG>::SMEM_BYTES, st, map_q, c, heads, topk, scale,
+    return launch_pdl(attend_kernel<HG>, grid, dim3(THREADS), Cfg<HG>::SMEM_BYTES, st, map_q, c, heads, topk, q, scale,
                       out, out_is_fp32, flags, lse);
 }
 

@@ -230,6 +230,28 @@ def test_step_is_repeatable_after_restore():
     assert torch.equal(a, dw.outs[0])
 
 
+def test_repeated_calls_leave_the_step_unchanged():
+    """The bench's marginal cost of a call makes every call of one kind twice
+    in place (csa2_attend; a Full layer's csa2_index; a Reindex layer's): each
+    repeat reads the same inputs and rewrites the same outputs, so every
+    layer's output and top-k stay bit-identical to the plain step's."""
+    w = synth.workload(3, small=True)
+    dw = DeviceWorkload(w, out_fp32=True)
+    dw.step()
+    torch.cuda.synchronize()
+    outs = [o.clone() for o in dw.outs]
+    tops = [t.clone() for t in dw.topk]
+    for kind in ("attend", "full", "reindex"):
+        dw.restore()
+        dw.step(repeat={kind: 2})
+        torch.cuda.synchronize()
+        assert csa2.csa2_get_device_error(dw.cache) == 0
+        for li, (a, o) in enumerate(zip(outs, dw.outs)):
+            assert torch.equal(a, o), f"{kind} repeated: layer {li} output differs"
+        for g, (a, t) in enumerate(zip(tops, dw.topk)):
+            assert torch.equal(a, t), f"{kind} repeated: top-k of group {g} differs"
+
+
 # ------------------------------------------------------------------ device-side data checks
 def test_bad_topk_index_sets_error_and_is_skipped():
     w = synth.workload(0, small=True)
