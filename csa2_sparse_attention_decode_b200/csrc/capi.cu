@@ -54,6 +54,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct Workspace {
     float *scores;
     int32_t *blocks;
+    uint4 *range;           // per request: the block scan's key range, folded by its CTAs
     int64_t row_stride;
     size_t bytes;
 };
@@ -66,6 +67,7 @@ Workspace layout(void *base, int32_t batch, int32_t max_entries)
     auto take = [&](size_t n) { size_t o = off; off = align256(off + n); return (char *)base + o; };
     w.scores = (float *)take(sizeof(float) * (size_t)batch * (size_t)w.row_stride);
     w.blocks = (int32_t *)take(sizeof(int32_t) * (size_t)batch * CSA2_MAX_BLOCKS);
+    w.range = (uint4 *)take(sizeof(uint4) * RANGE_SLOTS * (size_t)batch);
     w.bytes = off;
     return w;
 }
@@ -141,10 +143,11 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode, const uint
     }
     if (mode == CSA2_INDEX_FULL) {
         const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
-        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, W.scores, W.row_stride, s);
+        e = launch_score(c, ROWS_SUMMARIES, q_idx, w, W.scores, W.row_stride, s, W.range);
         if (e == cudaSuccess)
             e = launch_select(c, ROWS_SUMMARIES, W.scores, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS,
-                              W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, max_blocks, s);
+                              W.blocks, CSA2_MAX_BLOCKS, 1, pool, pool_len, max_blocks, s, nullptr, nullptr, 0,
+                              W.range);
         if (e != cudaSuccess) return from_cuda(e);
     }
     return from_cuda(launch_pool_select(c, q_idx, w, pool, pool_len, topk, s));
@@ -198,10 +201,11 @@ csa2_status csa2_shard_blocks(const csa2_cache *shard, const int32_t *entry_offs
     CacheView c = make_view(shard);
     cudaStream_t s = (cudaStream_t)stream;
     const int max_blocks = (max_entries + CSA2_BLOCK - 1) / CSA2_BLOCK;
-    cudaError_t e = launch_score(c, ROWS_SUMMARIES, q_idx, w, W.scores, W.row_stride, s);
+    cudaError_t e = launch_score(c, ROWS_SUMMARIES, q_idx, w, W.scores, W.row_stride, s, W.range);
     if (e == cudaSuccess)
         e = launch_select(c, ROWS_SUMMARIES, W.scores, W.row_stride, nullptr, nullptr, CSA2_MAX_BLOCKS, block_ids,
-                          CSA2_MAX_BLOCKS, 0, nullptr, nullptr, max_blocks, s, block_scores, entry_offset, 3);
+                          CSA2_MAX_BLOCKS, 0, nullptr, nullptr, max_blocks, s, block_scores, entry_offset, 3,
+                          W.range);
     return from_cuda(e);
 }
 

@@ -37,7 +37,7 @@ constexpr size_t SEL_SMEM = (size_t)(SEL_CAP + 2 * sel::CAND + 2 * sel::RANK_MAX
 template <int NC>
 __device__ __forceinline__ void select_body(CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,
                       const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
-                      int32_t *pool_len, float *vals, const int32_t *id_off, int id_shift)
+                      int32_t *pool_len, float *vals, const int32_t *id_off, int id_shift, uint4 *range)
 {
     extern __shared__ uint32_t dsm[];
     const int rank = (NC > 1) ? (int)cg::this_cluster().block_rank() : 0;
@@ -67,6 +67,22 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     bf.bits = bf.all_idx + sel::RANK_MAX;
     bf.bits_words = SEL_BITS;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
+    // The scan's range of the request's keys, when it kept one: then the
+    // selection needs no exchange between its CTAs to find it.
+    __shared__ uint32_t s_range[4];
+    const bool use_range = range != nullptr && n > k;
+    static_assert(RANGE_SLOTS == 32, "one slot per lane");
+    if (use_range && tid < 32) {
+        const uint4 r = range[(size_t)b * RANGE_SLOTS + tid];
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, r.x), mn = __reduce_min_sync(0xffffffffu, r.y);
+        const uint32_t lb = __reduce_min_sync(0xffffffffu, r.z);
+        if (tid == 0) {
+            s_range[0] = mn;                       // smallest key
+            s_range[1] = mx;                       // largest key
+            s_range[2] = lb;                       // smallest maximum of a 32-row group
+            s_range[3] = (uint32_t)((n + 31) / 32);    // 32-row groups, each with at least one key
+        }
+    }
     if (in_smem) {
         // 8 independent loads in flight per thread per round.
         for (int e0 = 0; e0 < cnt; e0 += 8 * SEL_THREADS) {
@@ -106,15 +122,20 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     o.vals = vals;
     o.id_off = id_off;
     o.id_shift = id_shift;
-    sel::select_core<NC, SEL_THREADS>(bf, b, n, chunk, lo, cnt, k, kmin, kmax, o);
+    sel::select_core<NC, SEL_THREADS>(bf, b, n, chunk, lo, cnt, k, kmin, kmax, o, use_range ? s_range : nullptr);
+    // Every CTA of the cluster read the range before the last cluster
+    // barrier: start the next scan's reduction from the empty range.
+    if (range != nullptr && rank == 0 && tid < RANGE_SLOTS)
+        range[(size_t)b * RANGE_SLOTS + tid] = make_uint4(0u, 0xffffffffu, 0xffffffffu, 0u);
 }
 
 #define CSA2_SELECT_ARGS                                                                                      \
     CacheView c, int src, const float *scores, int64_t score_stride, const int32_t *pool_len_in,               \
         const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool, int32_t *pool_len,    \
-        float *vals, const int32_t *id_off, int id_shift
+        float *vals, const int32_t *id_off, int id_shift, uint4 *range
 #define CSA2_SELECT_PASS \
-    c, src, scores, score_stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift
+    c, src, scores, score_stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift, \
+        range
 
 template <int NC>
 __global__ void __launch_bounds__(SEL_THREADS, 1) select_cluster_kernel(CSA2_SELECT_ARGS)
@@ -131,7 +152,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_cta_kernel(CSA2_SELECT_
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
                           int32_t *pool_len, int max_n, cudaStream_t st, float *vals, const int32_t *id_off,
-                          int id_shift)
+                          int id_shift, uint4 *range)
 {
     static DeviceOnce once;
     static int cluster_size[DeviceOnce::N] = {};
@@ -157,14 +178,15 @@ cudaError_t launch_select(const CacheView &c, int src, const float *scores, int6
     LaunchScope scope(CSA2_KERNEL_SELECT, st);
     if (max_n <= SEL_CAP)   // fits one CTA's shared memory: no cluster barriers on the path
         return launch_pdl(select_cta_kernel, dim3(1, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores, stride,
-                          pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift);
+                          pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift,
+                          range);
     if (nc == 16)
         return launch_pdl_cluster(select_cluster_kernel<16>, dim3(16, c.batch), dim3(SEL_THREADS), smem, st, 16, c,
                                   src, scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len,
-                                  vals, id_off, id_shift);
+                                  vals, id_off, id_shift, range);
     return launch_pdl_cluster(select_cluster_kernel<8>, dim3(8, c.batch), dim3(SEL_THREADS), smem, st, 8, c, src,
                               scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals,
-                              id_off, id_shift);
+                              id_off, id_shift, range);
 }
 
 }  // namespace csa2

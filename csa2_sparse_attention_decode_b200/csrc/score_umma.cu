@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "idx_query.cuh"
 #include "index.cuh"
+#include "select.cuh"
 #include "umma.cuh"
 
 namespace csa2 {
@@ -65,6 +66,7 @@ struct Params {
     const float *w;
     float *scores;
     int64_t stride;
+    uint4 *range;       // optional: per request and slot {max key, min key, min of the 32-row groups' maxima, -}
 };
 
 __device__ __forceinline__ int rows_of_req(const Params &p, int b)
@@ -374,10 +376,25 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
         const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
         int cur_b = -1;
         float wr[CSA2_IDX_HEADS];                                  // this request's w'
+        // The request's range over this warp's rows, folded into one of its
+        // slots once per request and warp (the slots spread the atomics: a
+        // few dozen per word).
+        uint32_t r_mx = 0u, r_mn = 0xffffffffu, r_lb = 0xffffffffu;
+        auto fold_range = [&](int b) {
+            if (p.range && b >= 0 && lane == 0 && r_mx >= r_mn) {
+                uint4 *r = p.range + (size_t)b * RANGE_SLOTS + ((blockIdx.x * 4 + warp) % RANGE_SLOTS);
+                atomicMax(&r->x, r_mx);
+                atomicMin(&r->y, r_mn);
+                atomicMin(&r->z, r_lb);
+            }
+            r_mx = 0u;
+            r_mn = r_lb = 0xffffffffu;
+        };
         for (int j = 0; j < n_items; ++j, it.next()) {
             if (it.b != cur_b) {
                 // New request.  Every MMA issued so far has completed (the
                 // previous epilogue waited for it), so the q buffer is free.
+                fold_range(cur_b);
                 cur_b = it.b;
                 iq_split(tid, p.q_idx, p.w, cur_b, qbuf, wq);
                 fence_proxy_async_smem();
@@ -407,8 +424,21 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
                                    acc[hh & 3]);
             const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             const int row = it.t * TILE + tid;
-            if (ok && row < it.rows) p.scores[(size_t)it.b * p.stride + row] = sc;
+            const bool valid = ok && row < it.rows;
+            if (valid) p.scores[(size_t)it.b * p.stride + row] = sc;
+            if (p.range) {
+                // this warp's 32 rows: their largest and smallest key
+                const uint32_t key = sel::ord_key(sc);
+                const uint32_t mx = __reduce_max_sync(0xffffffffu, valid ? key : 0u);
+                const uint32_t mn = __reduce_min_sync(0xffffffffu, valid ? key : 0xffffffffu);
+                if (mx >= mn) {
+                    r_mx = max(r_mx, mx);
+                    r_mn = min(r_mn, mn);
+                    r_lb = min(r_lb, mx);
+                }
+            }
         }
+        fold_range(cur_b);
     }
     fence_before_sync();
     __syncthreads();
@@ -437,7 +467,7 @@ bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows)
 }
 
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, float *scores,
-                         int64_t stride, cudaStream_t st)
+                         int64_t stride, cudaStream_t st, uint4 *range)
 {
     if (c.batch > MAX_BATCH || (src != ROWS_KEYS && src != ROWS_SUMMARIES)) return cudaErrorInvalidValue;
     static DeviceOnce once;
@@ -460,7 +490,7 @@ cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, con
     if (!make_plane_map(&maps.summ8, c.summ, np * 8, 8) || !make_plane_map(&maps.summ128, c.summ, np * 8, 128) ||
         !make_plane_map(&maps.keys64, c.keys, np * 64, 64) || !make_plane_map(&maps.keys128, c.keys, np * 64, 128))
         return cudaErrorInvalidValue;
-    Params p{c, src, q_idx, w, scores, stride};
+    Params p{c, src, q_idx, w, scores, stride, range};
     const int kid = src == ROWS_KEYS ? CSA2_KERNEL_FLAT_SCORE : CSA2_KERNEL_BLOCK_SCORE;
     const size_t smem = SMEM_BYTES + 8 * ((size_t)c.batch + 1);
     LaunchScope scope(kid, st);

@@ -102,9 +102,14 @@ __device__ __forceinline__ uint32_t scan256(uint32_t v, uint32_t *scratch)
 // with lo = rank*chunk.  kmin / kmax: this thread's min / max over the keys
 // it staged (any split of the range over the threads; a thread without keys
 // passes kmin = 0xffffffff, kmax = 0).  NT = threads per CTA (a multiple of 32, at least 256).
+// range (optional, the same in every CTA of the cluster): the cluster-wide
+// {min key, max key, a lower bound of the threshold, number of disjoint key
+// groups the bound is the smallest maximum of}, worked out by the caller;
+// then kmin / kmax are unused and the first exchange round is skipped.
 template <int NC, int NT>
 __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int chunk, int lo, int cnt, int k,
-                                            uint32_t kmin, uint32_t kmax, const Out &o)
+                                            uint32_t kmin, uint32_t kmax, const Out &o,
+                                            const uint32_t *range = nullptr)
 {
     constexpr int NW = NT / 32;
     __shared__ __align__(16) uint32_t hist[2][256];
@@ -136,54 +141,57 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kk;
     bool ranked = false;                                    // candidates were ranked directly
     if (!take_all) {
-        // Range of the keys that matter.  Every thread holding a key holds
-        // one >= its own maximum, so when at least kk threads hold keys, the
-        // smallest per-thread maximum lb is a lower bound of the threshold:
-        // keys below it never need resolving, however far below they lie.
-        const bool has = kmin <= kmax;
-        uint32_t klb = has ? kmax : 0xffffffffu;
-        uint32_t nthr = __popc(__ballot_sync(0xffffffffu, has));
+        if (!range) {                                       // the range from one exchange round
+            // Range of the keys that matter.  Every thread holding a key holds
+            // one >= its own maximum, so when at least kk threads hold keys, the
+            // smallest per-thread maximum lb is a lower bound of the threshold:
+            // keys below it never need resolving, however far below they lie.
+            const bool has = kmin <= kmax;
+            uint32_t klb = has ? kmax : 0xffffffffu;
+            uint32_t nthr = __popc(__ballot_sync(0xffffffffu, has));
 #pragma unroll
-        for (int off = 16; off; off >>= 1) {
-            kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
-            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
-            klb = min(klb, __shfl_xor_sync(0xffffffffu, klb, off));
-        }
-        if (lane == 0) {
-            wsum[wid][0] = kmin;
-            wsum[wid][1] = kmax;
-            wsum[wid][2] = klb;
-            wsum[wid][3] = nthr;
-        }
-        __syncthreads();
-        if (wid == 0) {
-            const bool in = lane < NW;
-            const uint32_t a = __reduce_min_sync(0xffffffffu, in ? wsum[lane][0] : 0xffffffffu);
-            const uint32_t z = __reduce_max_sync(0xffffffffu, in ? wsum[lane][1] : 0u);
-            const uint32_t l = __reduce_min_sync(0xffffffffu, in ? wsum[lane][2] : 0xffffffffu);
-            const uint32_t t = __reduce_add_sync(0xffffffffu, in ? wsum[lane][3] : 0u);
-            if (lane == 0) {
-                s_mm[0] = a;
-                s_mm[1] = z;
-                s_mm[2] = l;
-                s_mm[3] = t;
+            for (int off = 16; off; off >>= 1) {
+                kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+                kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+                klb = min(klb, __shfl_xor_sync(0xffffffffu, klb, off));
             }
-        }
-        csync();
-        if (wid == 0) {                                     // one 16-byte load per rank, reduced in the warp
-            uint4 v = make_uint4(0xffffffffu, 0u, 0xffffffffu, 0u);
-            if (lane < NC) v = *reinterpret_cast<const uint4 *>(remote(&s_mm[0], lane));
-            const uint32_t a = __reduce_min_sync(0xffffffffu, v.x), z = __reduce_max_sync(0xffffffffu, v.y);
-            const uint32_t l = __reduce_min_sync(0xffffffffu, v.z), t = __reduce_add_sync(0xffffffffu, v.w);
             if (lane == 0) {
-                s_g[0] = a;
-                s_g[1] = z;
-                s_g[2] = l;
-                s_g[3] = t;
+                wsum[wid][0] = kmin;
+                wsum[wid][1] = kmax;
+                wsum[wid][2] = klb;
+                wsum[wid][3] = nthr;
             }
+            __syncthreads();
+            if (wid == 0) {
+                const bool in = lane < NW;
+                const uint32_t a = __reduce_min_sync(0xffffffffu, in ? wsum[lane][0] : 0xffffffffu);
+                const uint32_t z = __reduce_max_sync(0xffffffffu, in ? wsum[lane][1] : 0u);
+                const uint32_t l = __reduce_min_sync(0xffffffffu, in ? wsum[lane][2] : 0xffffffffu);
+                const uint32_t t = __reduce_add_sync(0xffffffffu, in ? wsum[lane][3] : 0u);
+                if (lane == 0) {
+                    s_mm[0] = a;
+                    s_mm[1] = z;
+                    s_mm[2] = l;
+                    s_mm[3] = t;
+                }
+            }
+            csync();
+            if (wid == 0) {                                     // one 16-byte load per rank, reduced in the warp
+                uint4 v = make_uint4(0xffffffffu, 0u, 0xffffffffu, 0u);
+                if (lane < NC) v = *reinterpret_cast<const uint4 *>(remote(&s_mm[0], lane));
+                const uint32_t a = __reduce_min_sync(0xffffffffu, v.x), z = __reduce_max_sync(0xffffffffu, v.y);
+                const uint32_t l = __reduce_min_sync(0xffffffffu, v.z), t = __reduce_add_sync(0xffffffffu, v.w);
+                if (lane == 0) {
+                    s_g[0] = a;
+                    s_g[1] = z;
+                    s_g[2] = l;
+                    s_g[3] = t;
+                }
+            }
+            __syncthreads();
         }
-        __syncthreads();
-        const uint32_t gmin = s_g[0], gmax = s_g[1], glb = s_g[2], gthr = s_g[3];
+        const uint32_t gmin = range ? range[0] : s_g[0], gmax = range ? range[1] : s_g[1];
+        const uint32_t glb = range ? range[2] : s_g[2], gthr = range ? range[3] : s_g[3];
         const uint32_t low = gthr >= (uint32_t)kk ? glb : gmin;
         int hi = 32 - __clz(low ^ gmax);                    // bits [hi-1 .. 0] vary above `low`
         pmask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
@@ -346,6 +354,9 @@ __device__ __forceinline__ void select_core(const Bufs &bf, int b, int n, int ch
     };
     const uint32_t lt_mask = (1u << lane) - 1u;
     auto write_one = [&](int gi, uint32_t pos) {
+        // A range that does not hold the keys (one left by a scan that
+        // aborted) could choose more than kk: the slots bound the stores.
+        if (pos >= (uint32_t)kk) return;
         if (o.expand) {
             static_assert(CSA2_BLOCK == 8, "a block's entries are two int4");
             int32_t *dst = o.pool + (size_t)b * CSA2_POOL + (size_t)pos * CSA2_BLOCK;

@@ -41,8 +41,9 @@ def test_sizes(csa2):
     assert csa2.csa2_page_bytes() == 64 * 256 + 64 * 32 + 64 * 128 + 8 * 128 == 27648
     assert csa2.csa2_swa_bytes() == 128 * 512 + 128 * 4
     ws = csa2.csa2_workspace_bytes(4, 1 << 20)
-    need = 4 * (1 << 20) * 4 + 4 * 2048 * 4            # scan scores + selected blocks
-    assert need <= ws <= need + 2 * 256
+    # scan scores + selected blocks + the scan's key range per request
+    need = 4 * (1 << 20) * 4 + 4 * 2048 * 4 + 4 * 512
+    assert need <= ws <= need + 3 * 256
     assert csa2.csa2_workspace_bytes(0, 10) == 0
 
 

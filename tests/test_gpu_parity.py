@@ -252,6 +252,39 @@ def test_repeated_calls_leave_the_step_unchanged():
             assert torch.equal(a, t), f"{kind} repeated: top-k of group {g} differs"
 
 
+@pytest.mark.parametrize("fill", ["zeros", "ones", "random"])
+def test_index_exact_whatever_the_workspace_holds(fill):
+    """The workspace keeps, per request, the range of the block scan's keys
+    (folded by the scan, read and then reset by the selection).  Whatever the
+    words hold before a call only widens that range, so the selections and
+    outputs equal those of a workspace that held the empty range."""
+    w = synth.workload(3, small=True)
+    dw = DeviceWorkload(w, out_fp32=True)
+    dw.step()
+    torch.cuda.synchronize()
+    outs = [o.clone() for o in dw.outs]
+    tops = [t.clone() for t in dw.topk]
+    pools = dw.pool.clone()
+    ws = dw.ws.view(torch.uint8)
+    if fill == "zeros":
+        ws.zero_()
+    elif fill == "ones":
+        ws.fill_(0xFF)
+    else:
+        g = torch.Generator(device="cuda").manual_seed(7)
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda", generator=g))
+    for _ in range(2):                  # the second call starts from the range the first one reset
+        dw.restore()
+        dw.step()
+        torch.cuda.synchronize()
+        assert csa2.csa2_get_device_error(dw.cache) == 0
+        assert torch.equal(pools, dw.pool)
+        for li, (a, o) in enumerate(zip(outs, dw.outs)):
+            assert torch.equal(a, o), f"{fill}: layer {li} output differs"
+        for g_, (a, t) in enumerate(zip(tops, dw.topk)):
+            assert torch.equal(a, t), f"{fill}: top-k of group {g_} differs"
+
+
 # ------------------------------------------------------------------ device-side data checks
 def test_bad_topk_index_sets_error_and_is_skipped():
     w = synth.workload(0, small=True)
