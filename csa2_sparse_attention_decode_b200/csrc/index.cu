@@ -68,15 +68,23 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     bf.bits_words = SEL_BITS;
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     // The scan's range of the request's keys, when it kept one: then the
-    // selection needs no exchange between its CTAs to find it.
+    // selection needs no exchange between its CTAs to find it.  Slots that a
+    // selection has reset carry RANGE_TAG in their last word (the scan's
+    // atomics leave it alone); until every slot does (a fresh workspace),
+    // the exchange runs instead.  Every CTA of the cluster reads the same
+    // words and takes the same decision.
     __shared__ uint32_t s_range[4];
-    const bool use_range = range != nullptr && n > k;
+    __shared__ int s_use_range;
     static_assert(RANGE_SLOTS == 32, "one slot per lane");
-    if (use_range && tid < 32) {
-        const uint4 r = range[(size_t)b * RANGE_SLOTS + tid];
+    if (tid < 32) {
+        bool ok = range != nullptr && n > k;
+        uint4 r = make_uint4(0u, 0xffffffffu, 0xffffffffu, 0u);
+        if (ok) r = range[(size_t)b * RANGE_SLOTS + tid];
+        ok = __all_sync(0xffffffffu, ok && r.w == RANGE_TAG);
         const uint32_t mx = __reduce_max_sync(0xffffffffu, r.x), mn = __reduce_min_sync(0xffffffffu, r.y);
         const uint32_t lb = __reduce_min_sync(0xffffffffu, r.z);
         if (tid == 0) {
+            s_use_range = ok;
             s_range[0] = mn;                       // smallest key
             s_range[1] = mx;                       // largest key
             s_range[2] = lb;                       // smallest maximum of a 32-row group
@@ -122,11 +130,11 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
     o.vals = vals;
     o.id_off = id_off;
     o.id_shift = id_shift;
-    sel::select_core<NC, SEL_THREADS>(bf, b, n, chunk, lo, cnt, k, kmin, kmax, o, use_range ? s_range : nullptr);
+    sel::select_core<NC, SEL_THREADS>(bf, b, n, chunk, lo, cnt, k, kmin, kmax, o, s_use_range ? s_range : nullptr);
     // Every CTA of the cluster read the range before the last cluster
     // barrier: start the next scan's reduction from the empty range.
     if (range != nullptr && rank == 0 && tid < RANGE_SLOTS)
-        range[(size_t)b * RANGE_SLOTS + tid] = make_uint4(0u, 0xffffffffu, 0xffffffffu, 0u);
+        range[(size_t)b * RANGE_SLOTS + tid] = make_uint4(0u, 0xffffffffu, 0xffffffffu, RANGE_TAG);
 }
 
 #define CSA2_SELECT_ARGS                                                                                      \

@@ -21,15 +21,18 @@ bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows);
 // Row scores of the block summaries (src ROWS_SUMMARIES) or of the keys
 // (ROWS_KEYS) of every request into scores[b * stride + row].  With range,
 // also folds the keys into range[b * RANGE_SLOTS + s] = {largest key,
-// smallest key, smallest maximum of a 32-row group, -} (order-preserving
+// smallest key, smallest maximum of a 32-row group, tag} (order-preserving
 // keys, atomic max / min, each warp into one of the request's slots; the
-// words must hold the empty range {0, ~0, ~0, 0} or a wider one beforehand).
+// words must hold the empty range {0, ~0, ~0, tag} or a wider one
+// beforehand, as the selection leaves them).
 constexpr int RANGE_SLOTS = 32;
+constexpr uint32_t RANGE_TAG = 0x43534132u;     // the last word of a slot a selection reset
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, float *scores,
                          int64_t stride, cudaStream_t st, uint4 *range = nullptr);
 // Top-k selection of the rows' scores.  With range (the scan's, above), the
-// selection takes its bounds from there and then resets range[b] to the
-// empty range for the next scan.
+// selection takes its bounds from there when every slot of the request
+// carries the tag, and then resets the slots to the tagged empty range for
+// the next scan.
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
                           int32_t *pool_len, int max_n, cudaStream_t st, float *vals = nullptr,

@@ -139,8 +139,8 @@ size_t csa2_swa_bytes(void);    /* CSA2_SWA_BYTES  */
  * at most `max_entries` entries: the scan's row scores, the selected blocks
  * and 512 bytes per request for the range of the scan's scores (attention
  * needs none of it).  The range words are kept between calls: a fresh
- * workspace needs no initialisation (its first selection may take a few more
- * radix passes), and any call's results are exact whatever they hold.  0 for batch <= 0 or max_entries < 0.
+ * workspace needs no initialisation (its first selection finds the range
+ * itself), and any call's results are exact whatever they hold.  0 for batch <= 0 or max_entries < 0.
  * The caller allocates it (256-byte aligned) and may share one workspace
  * between calls that run in stream order. */
 size_t csa2_workspace_bytes(int32_t batch, int32_t max_entries);

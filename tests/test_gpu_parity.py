@@ -252,12 +252,13 @@ def test_repeated_calls_leave_the_step_unchanged():
             assert torch.equal(a, t), f"{kind} repeated: top-k of group {g} differs"
 
 
-@pytest.mark.parametrize("fill", ["zeros", "ones", "random"])
+@pytest.mark.parametrize("fill", ["zeros", "ones", "random", "random-tagged"])
 def test_index_exact_whatever_the_workspace_holds(fill):
     """The workspace keeps, per request, the range of the block scan's keys
-    (folded by the scan, read and then reset by the selection).  Whatever the
-    words hold before a call only widens that range, so the selections and
-    outputs equal those of a workspace that held the empty range."""
+    (folded by the scan, read and then reset to a tagged empty range by the
+    selection).  Untagged words are not used; tagged ones holding anything
+    else only widen the range.  Either way the selections and outputs equal
+    those of the steady state."""
     w = synth.workload(3, small=True)
     dw = DeviceWorkload(w, out_fp32=True)
     dw.step()
@@ -273,6 +274,8 @@ def test_index_exact_whatever_the_workspace_holds(fill):
     else:
         g = torch.Generator(device="cuda").manual_seed(7)
         ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda", generator=g))
+        if fill == "random-tagged":         # every 16-byte slot's last word is the reset tag
+            ws.view(torch.int32)[3::4] = 0x43534132
     for _ in range(2):                  # the second call starts from the range the first one reset
         dw.restore()
         dw.step()
