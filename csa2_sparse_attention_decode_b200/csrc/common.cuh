@@ -134,10 +134,10 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Whether `kernel` can run at least one cluster of cluster_x CTAs of this
-// shape on the current device (asked once per kernel and size by callers).
+// How many clusters of cluster_x CTAs of this shape `kernel` can have
+// resident at once on the current device (0 if none fits, or on error).
 template <typename... KArgs>
-inline bool cluster_fits(void (*kernel)(KArgs...), dim3 block, size_t smem, int cluster_x)
+inline int max_active_clusters(void (*kernel)(KArgs...), dim3 block, size_t smem, int cluster_x)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster_x, 1, 1);
@@ -153,9 +153,17 @@ inline bool cluster_fits(void (*kernel)(KArgs...), dim3 block, size_t smem, int 
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, (void *)kernel, &cfg) != cudaSuccess) {
         cudaGetLastError();
-        return false;
+        return 0;
     }
-    return n >= 1;
+    return n;
+}
+
+// Whether `kernel` can run at least one cluster of cluster_x CTAs of this
+// shape on the current device (asked once per kernel and size by callers).
+template <typename... KArgs>
+inline bool cluster_fits(void (*kernel)(KArgs...), dim3 block, size_t smem, int cluster_x)
+{
+    return max_active_clusters(kernel, block, smem, cluster_x) >= 1;
 }
 
 // ---------------------------------------------------------------- errors

@@ -16,10 +16,13 @@ namespace cg = cooperative_groups;
 namespace csa2 {
 
 // ------------------------------------------------------------------ top-k
-// Rows longer than one CTA holds run on a cluster of 16 CTAs (8 where the
-// device cannot schedule 16 of these CTAs in one cluster).
+// Each row runs on one CTA or on a cluster of 4, 8 or 16, chosen per launch
+// by a cost model: resident waves x (the exchange rounds' fixed cost + the
+// per-CTA key passes).
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_CAP = 32768;         // keys a CTA keeps in shared memory (128 KB)
+constexpr double SELECT_ROUNDS_US[4] = {2.0, 8.0, 9.0, 10.0};   // fixed cost for 1, 4, 8, 16 CTAs
+constexpr double SELECT_KEY_NS = 1.5;                            // per key a CTA holds
 constexpr int SEL_BITS = SEL_CAP / 32;
 constexpr size_t SEL_SMEM = (size_t)(SEL_CAP + 2 * sel::CAND + 2 * sel::RANK_MAX + SEL_BITS) * sizeof(uint32_t);
 
@@ -87,8 +90,9 @@ __device__ __forceinline__ void select_body(CacheView c, int src, const float *s
             s_use_range = ok;
             s_range[0] = mn;                       // smallest key
             s_range[1] = mx;                       // largest key
-            s_range[2] = lb;                       // smallest maximum of a 32-row group
-            s_range[3] = (uint32_t)((n + 31) / 32);    // 32-row groups, each with at least one key
+            const int g = range_group(n);
+            s_range[2] = lb;                       // smallest maximum of a group of g rows
+            s_range[3] = (uint32_t)((n + g - 1) / g);  // groups of g rows, each with at least one key
         }
     }
     if (in_smem) {
@@ -157,42 +161,83 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_cta_kernel(CSA2_SELECT_
 }
 
 // ------------------------------------------------------------------ launchers
+namespace {
+
+// CTAs per request for a selection over at most max_n rows: a cluster of
+// 16, 8 or 4 CTAs, or one CTA (no cluster barriers).  act[i]: how many
+// selections of 1, 4, 8 and 16 CTAs can be resident at once.
+int select_ctas(int batch, int max_n, const int act[4])
+{
+    static const int sizes[4] = {1, 4, 8, 16};
+    int best = 16;
+    double best_us = 1e30;
+    for (int i = 0; i < 4; ++i) {
+        const int nc = sizes[i];
+        const long long chunk = ((long long)max_n + nc - 1) / nc;
+        if (chunk > SEL_CAP || act[i] < 1) continue;
+        const long long waves = (batch + act[i] - 1) / act[i];
+        const double us = (double)waves * (SELECT_ROUNDS_US[i] + SELECT_KEY_NS * 1e-3 * (double)chunk);
+        if (us < best_us) {
+            best_us = us;
+            best = nc;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+
 cudaError_t launch_select(const CacheView &c, int src, const float *scores, int64_t stride, const int32_t *pool_len_in,
                           const int32_t *ids, int k, int32_t *out, int out_stride, int expand, int32_t *pool,
                           int32_t *pool_len, int max_n, cudaStream_t st, float *vals, const int32_t *id_off,
                           int id_shift, uint4 *range)
 {
     static DeviceOnce once;
-    static int cluster_size[DeviceOnce::N] = {};
+    static int active[DeviceOnce::N][4] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     const int smem = (int)SEL_SMEM;
     if (e == cudaSuccess)
         e = once.run(dev, [&] {
-            cudaError_t r = cudaFuncSetAttribute(select_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem);
+            cudaError_t r = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(select_cluster_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(select_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(select_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-            if (r == cudaSuccess)
-                r = cudaFuncSetAttribute(select_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (r == cudaSuccess)
-                cluster_size[dev] = cluster_fits(select_cluster_kernel<16>, dim3(SEL_THREADS), smem, 16) ? 16 : 8;
-            return r;
+            if (r != cudaSuccess) return r;
+            int per_sm = 0, sms = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_cta_kernel, SEL_THREADS, smem) !=
+                    cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+                cudaGetLastError();
+                per_sm = sms = 0;
+            }
+            active[dev][0] = per_sm * sms;
+            active[dev][1] = max_active_clusters(select_cluster_kernel<4>, dim3(SEL_THREADS), smem, 4);
+            active[dev][2] = max_active_clusters(select_cluster_kernel<8>, dim3(SEL_THREADS), smem, 8);
+            active[dev][3] = max_active_clusters(select_cluster_kernel<16>, dim3(SEL_THREADS), smem, 16);
+            return cudaSuccess;
         });
     if (e != cudaSuccess) return e;
-    const int nc = cluster_size[dev];
+    const int nc = select_ctas(c.batch, max_n, active[dev]);
     LaunchScope scope(CSA2_KERNEL_SELECT, st);
-    if (max_n <= SEL_CAP)   // fits one CTA's shared memory: no cluster barriers on the path
+    if (nc == 1)
         return launch_pdl(select_cta_kernel, dim3(1, c.batch), dim3(SEL_THREADS), smem, st, c, src, scores, stride,
                           pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals, id_off, id_shift,
                           range);
-    if (nc == 16)
-        return launch_pdl_cluster(select_cluster_kernel<16>, dim3(16, c.batch), dim3(SEL_THREADS), smem, st, 16, c,
-                                  src, scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len,
-                                  vals, id_off, id_shift, range);
-    return launch_pdl_cluster(select_cluster_kernel<8>, dim3(8, c.batch), dim3(SEL_THREADS), smem, st, 8, c, src,
+    if (nc == 4)
+        return launch_pdl_cluster(select_cluster_kernel<4>, dim3(4, c.batch), dim3(SEL_THREADS), smem, st, 4, c, src,
+                                  scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals,
+                                  id_off, id_shift, range);
+    if (nc == 8)
+        return launch_pdl_cluster(select_cluster_kernel<8>, dim3(8, c.batch), dim3(SEL_THREADS), smem, st, 8, c, src,
+                                  scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals,
+                                  id_off, id_shift, range);
+    return launch_pdl_cluster(select_cluster_kernel<16>, dim3(16, c.batch), dim3(SEL_THREADS), smem, st, 16, c, src,
                               scores, stride, pool_len_in, ids, k, out, out_stride, expand, pool, pool_len, vals,
                               id_off, id_shift, range);
 }

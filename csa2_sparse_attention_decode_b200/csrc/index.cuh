@@ -21,12 +21,20 @@ bool make_plane_map(CUtensorMap *m, void *base, long long rows, int box_rows);
 // Row scores of the block summaries (src ROWS_SUMMARIES) or of the keys
 // (ROWS_KEYS) of every request into scores[b * stride + row].  With range,
 // also folds the keys into range[b * RANGE_SLOTS + s] = {largest key,
-// smallest key, smallest maximum of a 32-row group, tag} (order-preserving
-// keys, atomic max / min, each warp into one of the request's slots; the
-// words must hold the empty range {0, ~0, ~0, tag} or a wider one
-// beforehand, as the selection leaves them).
+// smallest key, smallest maximum of a group of range_group(n) rows, tag}
+// (order-preserving keys, atomic max / min, each warp into one of the
+// request's slots; the words must hold the empty range {0, ~0, ~0, tag} or
+// a wider one beforehand, as the selection leaves them).
 constexpr int RANGE_SLOTS = 32;
 constexpr uint32_t RANGE_TAG = 0x43534132u;     // the last word of a slot a selection reset
+// Rows per group for the lower bound of a request of n rows: the largest of
+// 32, 16 and 8 that still gives at least CSA2_MAX_BLOCKS groups (each group
+// holds a key at least as large as the bound, so with that many groups the
+// bound is at most the top-2048 threshold); 8 when none does.
+__host__ __device__ __forceinline__ int range_group(int n)
+{
+    return n >= 32 * CSA2_MAX_BLOCKS ? 32 : n >= 16 * CSA2_MAX_BLOCKS ? 16 : 8;
+}
 cudaError_t launch_score(const CacheView &c, int src, const uint16_t *q_idx, const float *w, float *scores,
                          int64_t stride, cudaStream_t st, uint4 *range = nullptr);
 // Top-k selection of the rows' scores.  With range (the scan's, above), the

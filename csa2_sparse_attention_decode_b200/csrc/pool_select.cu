@@ -324,10 +324,10 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
                                const int32_t *pool_len, int32_t *topk, cudaStream_t st, float *topk_scores,
                                const int32_t *id_off)
 {
-    // 16 CTAs per request where the device can schedule such clusters
-    // (shorter per-CTA row ranges), else 8.
+    // 16 CTAs per request (shorter per-CTA row ranges) unless clusters of
+    // 8 need fewer waves of resident clusters for this batch.
     static DeviceOnce once;
-    static int cluster_size[DeviceOnce::N] = {};
+    static int active16[DeviceOnce::N] = {}, active8[DeviceOnce::N] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
@@ -339,12 +339,15 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
                                          (int)Layout<16>::SMEM_BYTES);
             if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-            if (r == cudaSuccess)
-                cluster_size[dev] = cluster_fits(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16) ? 16 : 8;
+            if (r == cudaSuccess) {
+                active16[dev] = max_active_clusters(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16);
+                active8[dev] = max_active_clusters(pool_select_kernel<8>, dim3(NT), Layout<8>::SMEM_BYTES, 8);
+            }
             return r;
         });
     if (e != cudaSuccess) return e;
-    const int nc = cluster_size[dev];
+    const int a16 = active16[dev], a8 = max(1, active8[dev]);
+    const int nc = (a16 >= 1 && (c.batch + a16 - 1) / a16 <= (c.batch + a8 - 1) / a8) ? 16 : 8;
     CUtensorMap map_keys8;
     if (!make_plane_map(&map_keys8, c.keys, (long long)c.n_pages * CSA2_PAGE_ENTRIES, CSA2_BLOCK))
         return cudaErrorInvalidValue;

@@ -427,14 +427,24 @@ score_umma_kernel(const __grid_constant__ PlaneMaps maps, Params p)
             const bool valid = ok && row < it.rows;
             if (valid) p.scores[(size_t)it.b * p.stride + row] = sc;
             if (p.range) {
-                // this warp's 32 rows: their largest and smallest key
-                const uint32_t key = sel::ord_key(sc);
-                const uint32_t mx = __reduce_max_sync(0xffffffffu, valid ? key : 0u);
+                // this warp's 32 rows: their largest and smallest key, and
+                // the smallest maximum of their groups of g rows that hold a
+                // key (g the same for the whole request)
+                const uint32_t key = valid ? sel::ord_key(sc) : 0u;
+                const uint32_t mx = __reduce_max_sync(0xffffffffu, key);
                 const uint32_t mn = __reduce_min_sync(0xffffffffu, valid ? key : 0xffffffffu);
+                const int g = range_group(it.rows);           // the same in every lane
+                uint32_t lb = mx;                             // g = 32: the warp is the group
+                if (g < 32) {
+                    uint32_t gm = key;
+                    for (int o = g >> 1; o; o >>= 1) gm = max(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+                    const bool lead = (lane & (g - 1)) == 0 && row < it.rows && ok;
+                    lb = __reduce_min_sync(0xffffffffu, lead ? gm : 0xffffffffu);
+                }
                 if (mx >= mn) {
                     r_mx = max(r_mx, mx);
                     r_mn = min(r_mn, mn);
-                    r_lb = min(r_lb, mx);
+                    r_lb = min(r_lb, lb);
                 }
             }
         }

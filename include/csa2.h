@@ -200,9 +200,10 @@ csa2_status csa2_index(const csa2_cache *cache, csa2_index_mode mode,
  * as indices in ascending order to out[b*k ..], -1 padded to k.
  *   scores f32 device [batch][stride]; n int32 device [batch], each in
  *   0..stride (values outside are clamped); k in 1..2048; out int32 device
- *   [batch][k].  Scores must not be NaN.  Rows of up to 32768 elements are
- *   selected by one CTA each, longer rows by a cluster of 16 CTAs (8 on a
- *   device that cannot schedule 16).  No workspace. */
+ *   [batch][k].  Scores must not be NaN.  Each row is selected by one
+ *   CTA or by a cluster of 4, 8 or 16 CTAs (each CTA holding up to 32768
+ *   elements), whichever a cost model of the batch's resident waves favours.
+ *   No workspace. */
 csa2_status csa2_topk(const float *scores, int64_t stride, const int32_t *n, int32_t batch, int32_t k,
                       int32_t *out, csa2_stream_t stream);
 
