@@ -105,8 +105,8 @@ def schedule_bytes(ws) -> dict:
 # the ncu captures summarised under profiles/, valid only while the kernel's
 # source is the one that was captured.
 KNOWN_TRAFFIC = {
-    "block_scan": {"bytes": 67_490_560 + 588_800, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
-                   "sha256": "5833231de81e1d8e21f6bad7c4162d487f314f041914bdc240b4db569dd70d63"},
+    "block_scan": {"bytes": 67_491_072 + 667_648, "source": "csa2_sparse_attention_decode_b200/csrc/score_umma.cu",
+                   "sha256": "2dc2384a162732e0be3768422c4d23299fa532a6fbc867ce4330f6ae96507e2b"},
     "attend": {"bytes": 1_553_536, "source": "csa2_sparse_attention_decode_b200/csrc/attend.cu",
                "sha256": "018ce55581bfed6bd02fdd7017dbe4fba80cc82a6fe04529727c08e4cfb343db"},
 }
