@@ -84,3 +84,13 @@ def test_topk_rows_past_cluster_shared_memory():
     # so the selection re-reads the scores from global memory
     r = _rng(600000)
     _run([r.standard_normal(600000).astype(np.float32), np.round(r.standard_normal(600000) * 2) / 2], 2048)
+
+
+@pytest.mark.parametrize("batch,n,k", [(2, 1000, 512), (32, 32768, 512), (8, 16384, 2048), (4, 131072, 2048)])
+def test_topk_batches_that_take_each_cluster_size(batch, n, k):
+    # the launch picks one CTA, or clusters of 4, 8 or 16 CTAs per row, from
+    # the batch and the row length (these four shapes take 1, 4, 8 and 16 on
+    # a B200); every shape must give the oracle's exact selection
+    r = _rng(batch * n + k)
+    rows = [np.round(r.standard_normal(n) * 64).astype(np.float32) / 64 for _ in range(batch)]
+    _run(rows, k)
