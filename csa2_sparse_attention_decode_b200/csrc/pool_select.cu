@@ -7,7 +7,8 @@
 // 2048 blocks x 8 positions = 16384 candidates; top_k 512; Full builds the
 // pool, Reindex searches inside it with its own query).
 //
-// One cluster of NC = 16 CTAs per request (8 where 16 cannot be scheduled).
+// One cluster of NC = 16 CTAs per request, or 8 when clusters of 8 need
+// fewer waves of resident clusters for the batch.
 // CTA r scores pool rows [r*chunk, r*chunk + chunk) (chunk a multiple of
 // 128, at most 16384 / NC) and keeps the
 // order-preserving keys of its scores in shared memory; the cluster then runs
