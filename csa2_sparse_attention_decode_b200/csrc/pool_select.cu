@@ -7,8 +7,8 @@
 // 2048 blocks x 8 positions = 16384 candidates; top_k 512; Full builds the
 // pool, Reindex searches inside it with its own query).
 //
-// One cluster of NC = 16 CTAs per request, or 8 when clusters of 8 need
-// fewer waves of resident clusters for the batch.
+// One cluster of NC = 16, 8 or 4 CTAs per request, chosen per launch from
+// the batch and how many clusters of each size can be resident at once.
 // CTA r scores pool rows [r*chunk, r*chunk + chunk) (chunk a multiple of
 // 128, at most 16384 / NC) and keeps the
 // order-preserving keys of its scores in shared memory; the cluster then runs
@@ -50,7 +50,7 @@ constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;         // 16 KB
 // Shared-memory layout for NC CTAs per request (rows per CTA at most POOL/NC).
 template <int NC>
 struct Layout {
-    static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 2048 (NC = 8) or 1024 (NC = 16) rows
+    static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 4096, 2048 or 1024 rows (NC = 4, 8, 16)
     static constexpr int RUNS = CHUNK_MAX / CSA2_BLOCK;  // runs of 8 rows
     static constexpr int BITS_WORDS = CHUNK_MAX / 32;
     static constexpr size_t OFF_Q = (size_t)STAGES * STAGE_BYTES;
@@ -325,36 +325,53 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
                                const int32_t *pool_len, int32_t *topk, cudaStream_t st, float *topk_scores,
                                const int32_t *id_off)
 {
-    // 16 CTAs per request (shorter per-CTA row ranges) unless clusters of
-    // 8 need fewer waves of resident clusters for this batch.
+    // Clusters of 16, 8 or 4 CTAs per request, whichever minimises resident
+    // waves x a cluster's time (the selection's fixed ~12 us + ~0.74 us per
+    // gathered 128-row tile of a CTA, up to 16384 / NC rows).
     static DeviceOnce once;
-    static int active16[DeviceOnce::N] = {}, active8[DeviceOnce::N] = {};
+    static int active[DeviceOnce::N][3] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
         e = once.run(dev, [&] {
-            cudaError_t r = cudaFuncSetAttribute(pool_select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)Layout<8>::SMEM_BYTES);
+            cudaError_t r = cudaFuncSetAttribute(pool_select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)Layout<4>::SMEM_BYTES);
+            if (r == cudaSuccess)
+                r = cudaFuncSetAttribute(pool_select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Layout<8>::SMEM_BYTES);
             if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Layout<16>::SMEM_BYTES);
             if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (r == cudaSuccess) {
-                active16[dev] = max_active_clusters(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16);
-                active8[dev] = max_active_clusters(pool_select_kernel<8>, dim3(NT), Layout<8>::SMEM_BYTES, 8);
+                active[dev][0] = max_active_clusters(pool_select_kernel<4>, dim3(NT), Layout<4>::SMEM_BYTES, 4);
+                active[dev][1] = max_active_clusters(pool_select_kernel<8>, dim3(NT), Layout<8>::SMEM_BYTES, 8);
+                active[dev][2] = max_active_clusters(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16);
             }
             return r;
         });
     if (e != cudaSuccess) return e;
-    const int a16 = active16[dev], a8 = max(1, active8[dev]);
-    const int nc = (a16 >= 1 && (c.batch + a16 - 1) / a16 <= (c.batch + a8 - 1) / a8) ? 16 : 8;
+    int nc = 8;
+    double best = 1e30;
+    for (int i = 2; i >= 0; --i) {                  // 16 first: it wins ties
+        const int size = 4 << i, act = active[dev][i];
+        if (act < 1) continue;
+        const double us = (double)((c.batch + act - 1) / act) * (12.0 + 0.74 * (CSA2_POOL / size / TILE));
+        if (us < best) {
+            best = us;
+            nc = size;
+        }
+    }
     CUtensorMap map_keys8;
     if (!make_plane_map(&map_keys8, c.keys, (long long)c.n_pages * CSA2_PAGE_ENTRIES, CSA2_BLOCK))
         return cudaErrorInvalidValue;
     LaunchScope scope(CSA2_KERNEL_POOL_SCORE, st);
     if (nc == 16)
         return launch_pdl_cluster(pool_select_kernel<16>, dim3(16, c.batch), dim3(NT), Layout<16>::SMEM_BYTES, st, 16,
+                                  map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
+    if (nc == 4)
+        return launch_pdl_cluster(pool_select_kernel<4>, dim3(4, c.batch), dim3(NT), Layout<4>::SMEM_BYTES, st, 4,
                                   map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
     return launch_pdl_cluster(pool_select_kernel<8>, dim3(8, c.batch), dim3(NT), Layout<8>::SMEM_BYTES, st, 8,
                               map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
