@@ -158,14 +158,6 @@ inline int max_active_clusters(void (*kernel)(KArgs...), dim3 block, size_t smem
     return n;
 }
 
-// Whether `kernel` can run at least one cluster of cluster_x CTAs of this
-// shape on the current device (asked once per kernel and size by callers).
-template <typename... KArgs>
-inline bool cluster_fits(void (*kernel)(KArgs...), dim3 block, size_t smem, int cluster_x)
-{
-    return max_active_clusters(kernel, block, smem, cluster_x) >= 1;
-}
-
 // ---------------------------------------------------------------- errors
 __device__ __forceinline__ void set_error(int32_t *err, int32_t code)
 {
