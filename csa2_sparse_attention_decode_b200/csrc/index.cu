@@ -165,11 +165,13 @@ namespace {
 
 // CTAs per request for a selection over at most max_n rows: a cluster of
 // 16, 8 or 4 CTAs, or one CTA (no cluster barriers).  act[i]: how many
-// selections of 1, 4, 8 and 16 CTAs can be resident at once.
+// selections of 1, 4, 8 and 16 CTAs can be resident at once.  Rows longer
+// than any size keeps in shared memory take the largest cluster the device
+// can run (its CTAs then re-read the scores from global memory).
 int select_ctas(int batch, int max_n, const int act[4])
 {
     static const int sizes[4] = {1, 4, 8, 16};
-    int best = 16;
+    int best = act[3] >= 1 ? 16 : act[2] >= 1 ? 8 : 4;
     double best_us = 1e30;
     for (int i = 0; i < 4; ++i) {
         const int nc = sizes[i];
