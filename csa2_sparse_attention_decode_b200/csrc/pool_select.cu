@@ -7,8 +7,8 @@
 // 2048 blocks x 8 positions = 16384 candidates; top_k 512; Full builds the
 // pool, Reindex searches inside it with its own query).
 //
-// One cluster of NC = 16, 8 or 4 CTAs per request, chosen per launch from
-// the batch and how many clusters of each size can be resident at once.
+// One cluster of NC = 16, 8, 4 or 2 CTAs per request, chosen per launch
+// from the batch and how many clusters of each size can be resident at once.
 // CTA r scores pool rows [r*chunk, r*chunk + chunk) (chunk a multiple of
 // 128, at most 16384 / NC) and keeps the
 // order-preserving keys of its scores in shared memory; the cluster then runs
@@ -50,7 +50,7 @@ constexpr int STAGE_BYTES = TILE * CSA2_KEY_DIM;         // 16 KB
 // Shared-memory layout for NC CTAs per request (rows per CTA at most POOL/NC).
 template <int NC>
 struct Layout {
-    static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 4096, 2048 or 1024 rows (NC = 4, 8, 16)
+    static constexpr int CHUNK_MAX = CSA2_POOL / NC;     // 8192 ... 1024 rows (NC = 2 ... 16)
     static constexpr int RUNS = CHUNK_MAX / CSA2_BLOCK;  // runs of 8 rows
     static constexpr int BITS_WORDS = CHUNK_MAX / 32;
     static constexpr size_t OFF_Q = (size_t)STAGES * STAGE_BYTES;
@@ -325,15 +325,20 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
                                const int32_t *pool_len, int32_t *topk, cudaStream_t st, float *topk_scores,
                                const int32_t *id_off)
 {
-    // Clusters of 16, 8 or 4 CTAs per request, whichever minimises resident
-    // waves x a cluster's time (the selection's fixed ~12 us + ~0.74 us per
-    // gathered 128-row tile of a CTA, up to 16384 / NC rows).
+    // Clusters of 16, 8, 4 or 2 CTAs per request, whichever minimises
+    // resident waves x a cluster's time (the selection's fixed ~12 us +
+    // ~0.74 us per gathered 128-row tile of a CTA, up to 16384 / NC rows).
     static DeviceOnce once;
-    static int active[DeviceOnce::N][3] = {};
+    static int active[DeviceOnce::N][4] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
         e = once.run(dev, [&] {
+            // Clusters of 2 need nearly all of a CTA's shared memory: left out
+            // where the device does not grant it.
+            const bool two = cudaFuncSetAttribute(pool_select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  (int)Layout<2>::SMEM_BYTES) == cudaSuccess;
+            if (!two) cudaGetLastError();
             cudaError_t r = cudaFuncSetAttribute(pool_select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)Layout<4>::SMEM_BYTES);
             if (r == cudaSuccess)
@@ -345,17 +350,18 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
             if (r == cudaSuccess)
                 r = cudaFuncSetAttribute(pool_select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (r == cudaSuccess) {
-                active[dev][0] = max_active_clusters(pool_select_kernel<4>, dim3(NT), Layout<4>::SMEM_BYTES, 4);
-                active[dev][1] = max_active_clusters(pool_select_kernel<8>, dim3(NT), Layout<8>::SMEM_BYTES, 8);
-                active[dev][2] = max_active_clusters(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16);
+                active[dev][0] = two ? max_active_clusters(pool_select_kernel<2>, dim3(NT), Layout<2>::SMEM_BYTES, 2) : 0;
+                active[dev][1] = max_active_clusters(pool_select_kernel<4>, dim3(NT), Layout<4>::SMEM_BYTES, 4);
+                active[dev][2] = max_active_clusters(pool_select_kernel<8>, dim3(NT), Layout<8>::SMEM_BYTES, 8);
+                active[dev][3] = max_active_clusters(pool_select_kernel<16>, dim3(NT), Layout<16>::SMEM_BYTES, 16);
             }
             return r;
         });
     if (e != cudaSuccess) return e;
     int nc = 8;
     double best = 1e30;
-    for (int i = 2; i >= 0; --i) {                  // 16 first: it wins ties
-        const int size = 4 << i, act = active[dev][i];
+    for (int i = 3; i >= 0; --i) {                  // 16 first: it wins ties
+        const int size = 2 << i, act = active[dev][i];
         if (act < 1) continue;
         const double us = (double)((c.batch + act - 1) / act) * (12.0 + 0.74 * (CSA2_POOL / size / TILE));
         if (us < best) {
@@ -369,6 +375,9 @@ cudaError_t launch_pool_select(const CacheView &c, const uint16_t *q_idx, const 
     LaunchScope scope(CSA2_KERNEL_POOL_SCORE, st);
     if (nc == 16)
         return launch_pdl_cluster(pool_select_kernel<16>, dim3(16, c.batch), dim3(NT), Layout<16>::SMEM_BYTES, st, 16,
+                                  map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
+    if (nc == 2)
+        return launch_pdl_cluster(pool_select_kernel<2>, dim3(2, c.batch), dim3(NT), Layout<2>::SMEM_BYTES, st, 2,
                                   map_keys8, c, q_idx, w, pool, pool_len, topk, topk_scores, id_off);
     if (nc == 4)
         return launch_pdl_cluster(pool_select_kernel<4>, dim3(4, c.batch), dim3(NT), Layout<4>::SMEM_BYTES, st, 4,
